@@ -1,0 +1,60 @@
+"""Plants plausible mistakes in copies of the oracle and requires the pins to catch each.
+
+Every mutant below is a one-line edit of oracle/hs2_oracle.cpp (a dropped term, a wrong
+sign, index or bound, a swapped operand).  The test compiles the edited copy in a
+temporary directory, routes the oracle wrapper to it and runs every pin; at least one
+pin must fail.  Nothing here touches a GPU.
+"""
+
+import os
+
+import pytest
+
+import oracle
+import oracle_pins as P
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "hs2_oracle.cpp")
+
+MUTANTS = {
+    "logit_scale_dropped": ("p[(size_t)h * n + j] = scale * acc;", "p[(size_t)h * n + j] = acc;"),
+    "softmax_max_not_subtracted": ("ph[j] = std::exp(ph[j] - m) / l;", "ph[j] = std::exp(ph[j]) / l;"),
+    "lse_wrong": ("lse_row[h] = m + std::log(l);", "lse_row[h] = m + l;"),
+    "score_not_head_summed": ("s += pj;", "s = pj;"),
+    "window_short_by_one": ("for (int64_t j = std::max<int64_t>(0, i - window + 1); j <= i; ++j) sel.push_back(j);",
+                            "for (int64_t j = std::max<int64_t>(0, i - window + 2); j <= i; ++j) sel.push_back(j);"),
+    "candidates_overlap_window": ("for (int64_t j = 0; j <= i - window; ++j) cand.push_back(j);",
+                                  "for (int64_t j = 0; j <= i - window + 1; ++j) cand.push_back(j);"),
+    "ties_to_higher_index": ("return a < b;", "return a > b;"),
+    "scores_ascending": ("if (score[a] != score[b]) return score[a] > score[b];",
+                         "if (score[a] != score[b]) return score[a] < score[b];"),
+    "query_position_ignores_offset": ("int64_t i = L - T + t, n = i + 1;", "int64_t i = t + (L > T ? 1 : 0), n = i + 1;"),
+    "bridge_operand_transposed": ("acc += xd[k] * bf16_to_f64(w[k]);",
+                                  "acc += xd[k] * bf16_to_f64(Wt[((int64_t)k * n_cols + c) % ((int64_t)n_cols * hidden)]);"),
+    "fp8_scale_wrong_max": ("double s = amax > 0.0 ? amax / 448.0 : 1.0;", "double s = amax > 0.0 ? amax / 240.0 : 1.0;"),
+    "e4m3_bias_wrong": ("(1.0 + m / 8.0) * std::ldexp(1.0, e - 7);", "(1.0 + m / 8.0) * std::ldexp(1.0, e - 8);"),
+    "e4m3_ties_to_odd": ("(d == best_d && (c % 2) == 0)", "(d == best_d && (c % 2) == 1)"),
+    "bf16_truncates": ("double r = std::nearbyint(x / ulp) * ulp;", "double r = std::trunc(x / ulp) * ulp;"),
+    "sparse_uses_v_as_k": ("kd[(size_t)n * D + d] = kv.key(b, sel[n], d);", "kd[(size_t)n * D + d] = kv.val(b, sel[n], d);"),
+    "sparse_softmax_not_normalised": ("for (int n = 0; n < ns; ++n) pr[n] = std::exp(pr[n] - m) / l;",
+                                      "for (int n = 0; n < ns; ++n) pr[n] = std::exp(pr[n] - m);"),
+    "fp8_value_scale_ignored": ("if (fp8) return e4m3_to_f64(((const uint8_t*)base)[off]) * (double)sc[(int64_t)b * L + j];",
+                                "if (fp8) return e4m3_to_f64(((const uint8_t*)base)[off]) * (double)sc[(int64_t)b * L];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, "mutation site not found exactly once: " + name
+    path = tmp_path / "mutant.cpp"
+    path.write_text(src.replace(old, new))
+    lib = oracle.compile_source(str(path), str(tmp_path / "libmutant.so"))
+    caught = []
+    with oracle.use_library(lib):
+        for check in P.ALL_CHECKS:
+            try:
+                check()
+            except AssertionError:
+                caught.append(check.__name__)
+    assert caught, "no pin caught mutant " + name
