@@ -1,0 +1,182 @@
+/*
+ * hs2.h -- C ABI of libhs2, the B200 (sm_100a) hot path of the HySparse2
+ * Cross-Decoder hybrid block.
+ *
+ * The HySparse2 pages describe a model split into a Self-Decoder and a
+ * Cross-Decoder joined by two levels of KV sharing (IT Home announcement of
+ * MiMo HySparse2, the "KV Bridging" / "KV Reuse" paragraphs; toolnavs.com
+ * summary, section "HySparse2 がやったこと"):
+ *   1. KV Bridging: every full-attention layer of the Cross-Decoder builds its
+ *      own K/V cache from the input hidden state of the corresponding
+ *      Self-Decoder full-attention layer, with its own K/V projection.
+ *   2. KV Reuse: inside a hybrid block (one full-attention layer followed by
+ *      several sparse-attention layers), the full-attention layer selects
+ *      important positions from its attention scores while it computes, and
+ *      the sparse layers reuse its KV cache and those indices.
+ *   Selection is per token: the 128 most recent tokens are always taken, and
+ *   1024 global tokens are chosen from outside that window (IT Home
+ *   announcement, token-level selection paragraph; cnyes.com article, section
+ *   "檢索精確到token").
+ *
+ * The three compute entry points below are those three steps.  The pages give
+ * no formulas; the readings this library takes are stated at each function.
+ *
+ * Conventions (all functions):
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The
+ *     library allocates no device or host memory; scratch comes from the
+ *     caller's workspace, sized by the matching *_workspace() function.
+ *   - Work is enqueued on `stream` and the call returns without waiting.
+ *     Arguments are checked on the host before anything is enqueued; a bad
+ *     argument returns HS2_ERR_INVALID_ARG and enqueues nothing.  A shape the
+ *     kernels do not implement returns HS2_ERR_UNSUPPORTED.  A failed launch
+ *     returns HS2_ERR_CUDA.  The library never aborts or exits.
+ *   - Kernels that wait on on-chip barriers give up after about one second,
+ *     set a bit in a per-device status word and return; read and clear it
+ *     with hs2_last_device_status().
+ *   - Pointers must be 16-byte aligned.  bf16 is IEEE binary32's upper half;
+ *     E4M3 is the OCP 8-bit float (bias 7, max 448, no infinities).
+ *   - MQA cache layout: one KV head.  For B sequences of L positions, K and V
+ *     are [B][L][D] row-major (bf16: 2 bytes, E4M3: 1 byte per element); for
+ *     E4M3, k_scale and v_scale are fp32 [B][L] and the stored value of
+ *     element d of position j is e4m3(code) * scale[j].
+ */
+#ifndef HS2_H
+#define HS2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define HS2_API __attribute__((visibility("default")))
+#else
+#define HS2_API
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* hs2_stream_t;
+
+typedef enum {
+  HS2_OK = 0,
+  HS2_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, inconsistent sizes  */
+  HS2_ERR_UNSUPPORTED = 2,  /* valid request, shape not implemented         */
+  HS2_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed         */
+  HS2_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than required      */
+  HS2_ERR_TIMEOUT = 5,      /* a kernel gave up waiting on a barrier        */
+  HS2_ERR_DEVICE = 6        /* a kernel found an out-of-range index         */
+} hs2_status;
+
+typedef enum { HS2_KV_BF16 = 0, HS2_KV_FP8_E4M3 = 1 } hs2_kv_dtype;
+
+/* One layer's MQA cache: device pointers.  Scales are NULL for bf16. */
+typedef struct {
+  void* k;
+  void* v;
+  float* k_scale;
+  float* v_scale;
+} hs2_kv_cache;
+
+/*
+ * hs2_bridge_kv -- KV Bridging (IT Home announcement, "KV Bridging"
+ * paragraph; toolnavs.com summary: each target layer has its own K/V
+ * projection of the same source hidden state).
+ *
+ * For every target layer l in [0, n_layers) and token r in [0, T):
+ *   K_l[r][d] = sum_k X[r][k] * Wt[l*2*D + d][k]
+ *   V_l[r][d] = sum_k X[r][k] * Wt[l*2*D + D + d][k]
+ * computed as one GEMM Y = X * Wt^T with fp32 accumulation.
+ *   X   : bf16 [T][hidden] row-major (the source layer's input hidden state).
+ *   Wt  : bf16 [n_layers*2*D][hidden] row-major; row c holds the weights of
+ *         output column c (nn.Linear weight layout).
+ *   caches[l] (host array of n_layers structs of device pointers): rows
+ *         cache_row_offset .. cache_row_offset+T-1 of K_l and V_l are written.
+ *   out_dtype HS2_KV_BF16: K, V bf16 [rows][D] (round to nearest even).
+ *   out_dtype HS2_KV_FP8_E4M3: per token and tensor, s = max_d |Y| / 448
+ *         (s = 1 when the row is all zero) is written to k_scale/v_scale[row]
+ *         and the codes E4M3(Y / s) (round to nearest even, saturating) to
+ *         K/V [rows][D].
+ * Supported: D == 128, hidden % 64 == 0, hidden >= 64, n_layers >= 1.
+ */
+HS2_API hs2_status hs2_bridge_kv(const void* X, int64_t T, int hidden, const void* Wt, int n_layers,
+                         int D, hs2_kv_dtype out_dtype, const hs2_kv_cache* caches,
+                         int64_t cache_row_offset, hs2_stream_t stream);
+
+/*
+ * Workspace bytes needed by hs2_full_attn_select for these sizes.
+ * Returns 0 for arguments hs2_full_attn_select would reject.
+ */
+HS2_API size_t hs2_full_attn_select_workspace(int B, int T, int64_t L, int H, int D, int topk,
+                                      int window, hs2_kv_dtype dt);
+
+/*
+ * hs2_full_attn_select -- the hybrid block's full-attention layer and its
+ * token selection (IT Home announcement, "KV Reuse" paragraphs: the full
+ * layer picks important positions from its attention scores; token-level
+ * selection paragraph: 128 most recent tokens forced, 1024 more from outside
+ * that window).
+ *
+ * Query t of sequence b sits at position i = L - T + t of that sequence's
+ * cache (the cache already holds the queries' own tokens).  For head h:
+ *   s_hj   = scale * <Q[b][t][h], K[b][j]>          for j <= i (causal)
+ *   p_hj   = exp(s_hj - lse_h),  lse_h = log sum_{j<=i} exp(s_hj)
+ *   O[b][t][h][d] = sum_j p_hj V[b][j][d]
+ * Selection (readings of this library where the pages are silent):
+ *   score_j = sum_h p_hj (head-summed softmax probability);
+ *   candidates C = {0 .. i-window}; window W = {max(0,i-window+1) .. i};
+ *   S = W  union  the min(topk, |C|) candidates of largest score, ties to
+ *   the lower position.
+ * Outputs:
+ *   O     : fp32 [B][T][H][D].
+ *   lse   : fp32 [B][T][H] natural-log normaliser, or NULL.
+ *   idx   : int32 [B][T][topk+window]: S in ascending order, then -1 padding.
+ *   n_sel : int32 [B][T]: |S| = min(topk, |C|) + min(window, i+1).
+ * Inputs: Q bf16 [B][T][H][D]; kv points to one hs2_kv_cache (host struct).
+ * Supported: D in {64, 128}; H in {8, 16, 32}; 1 <= T <= L; L < 2^31;
+ * 0 <= topk; 1 <= window; topk + window <= 4096.
+ */
+HS2_API hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, int T, int64_t L,
+                                int H, int D, float scale, int topk, int window,
+                                hs2_kv_dtype dt, float* O, float* lse, int32_t* idx,
+                                int32_t* n_sel, void* workspace, size_t workspace_bytes,
+                                hs2_stream_t stream);
+
+/*
+ * hs2_sparse_attn -- a sparse-attention layer with KV Reuse (IT Home
+ * announcement, "KV Reuse" paragraph: the sparse layers reuse the full
+ * layer's KV cache and selection indices; the SWA branch is folded into the
+ * forced window, so there is no second cache).
+ *
+ * For each query (b, t) and head h, over the positions S = idx[b][t][0 ..
+ * n_sel[b][t]) of the same cache, softmax renormalised over S only:
+ *   O[b][t][h][d] = sum_{j in S} softmax_j(scale * <Q[b][t][h], K[b][j]>) V[b][j][d]
+ * Q is this layer's own bf16 [B][T][H][D]; idx/n_sel as written by
+ * hs2_full_attn_select, with `slots` entries per query (>= n_sel).  Entries
+ * outside [0, L) raise HS2_ERR_DEVICE through hs2_last_device_status and are
+ * skipped.  A query with n_sel == 0 gets O = 0.
+ * Supported: D in {64, 128}; H in {8, 16, 32}; slots <= 4096.
+ */
+HS2_API hs2_status hs2_sparse_attn(const void* Q, const hs2_kv_cache* kv, int B, int T, int64_t L, int H,
+                           int D, float scale, const int32_t* idx, const int32_t* n_sel,
+                           int slots, hs2_kv_dtype dt, float* O, hs2_stream_t stream);
+
+/*
+ * Waits for `stream`, then reads and clears the calling device's status
+ * word: HS2_OK, HS2_ERR_TIMEOUT (a barrier wait gave up) or HS2_ERR_DEVICE
+ * (an index was out of range).  HS2_ERR_CUDA if the wait itself failed.
+ */
+HS2_API hs2_status hs2_last_device_status(hs2_stream_t stream);
+
+/* Static English description of a status code. */
+HS2_API const char* hs2_status_string(hs2_status status);
+
+/* Library ABI version: 100 * major + minor. */
+HS2_API int hs2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HS2_H */

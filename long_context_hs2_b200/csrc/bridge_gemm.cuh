@@ -1,0 +1,277 @@
+// KV Bridging GEMM on the 5th-generation tensor cores (tcgen05).
+//
+// Y = X * Wt^T, X [T][hidden] bf16, Wt [n_layers*256][hidden] bf16 (D = 128:
+// every target layer owns 256 output columns, K_l then V_l).  One output tile
+// is 128 tokens x 256 columns = one layer's K and V for 128 tokens, so the
+// epilogue thread that owns a token row sees all 128 values of K_l (and of
+// V_l) and computes the per-token E4M3 scale without any cross-thread step.
+//
+// Persistent kernel, one CTA per SM, 6 warps:
+//   warp 0      TMA producer: 64-wide K slices of X (128 rows) and Wt (256
+//               rows), 128B-swizzled, into a 4-stage ring (48 KB per stage).
+//   warp 1      TMEM allocator and MMA issuer: one thread issues
+//               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) x 4 per
+//               stage into a fp32 accumulator in tensor memory; tcgen05.commit
+//               releases ring stages and publishes finished accumulators.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//               32*(w%4) .. +31 = its 32 token rows), conversion to bf16 or to
+//               E4M3 + per-token scale, stores to the per-layer caches.
+// The accumulator is double-buffered (2 x 256 of the 512 TMEM columns) so the
+// epilogue of tile i overlaps the MMAs of tile i+1.
+#pragma once
+
+#include "hs2_common.cuh"
+
+namespace hs2 {
+
+constexpr int kBrMaxLayers = 16;
+constexpr int kBrBM = 128, kBrBN = 256, kBrBK = 64;
+constexpr int kBrStages = 4;
+constexpr int kBrABytes = kBrBM * kBrBK * 2;   // 16 KB
+constexpr int kBrBBytes = kBrBN * kBrBK * 2;   // 32 KB
+constexpr int kBrStageBytes = kBrABytes + kBrBBytes;
+constexpr int kBrBarOff = kBrStages * kBrStageBytes;
+constexpr int kBrSmemBytes = kBrBarOff + 256 + 1024;
+constexpr int kBrThreads = 192;
+
+struct BridgeParams {
+  void* k[kBrMaxLayers];
+  void* v[kBrMaxLayers];
+  float* k_scale[kBrMaxLayers];
+  float* v_scale[kBrMaxLayers];
+  long long T;
+  long long row_offset;
+  int hidden, n_layers, fp8;
+};
+
+// ---------------------------------------------------------- tcgen05 PTX --
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+// Arrives once on `bar` when every tcgen05.mma issued so far by this thread completes.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulator.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes (one lane per thread).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand tile stored as rows of
+// 128 bytes (64 bf16) with the 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);         // start address
+  d |= (uint64_t)1u << 16;                         // leading byte offset (unused here)
+  d |= (uint64_t)(1024u >> 4) << 32;               // stride byte offset: 8 rows
+  d |= (uint64_t)1u << 46;                         // descriptor version (sm_100)
+  d |= (uint64_t)2u << 61;                         // layout: 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: kind::f16, A = B = bf16, D = fp32, both K-major.
+__host__ __device__ constexpr uint32_t bridge_idesc() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBrBN >> 3) << 17) |
+         ((uint32_t)(kBrBM >> 4) << 24);
+}
+
+// Epilogue for one 128-column half (K or V) of a token row: v[128] fp32.
+__device__ __forceinline__ void bridge_store_row(const BridgeParams& p, int layer, int kv,
+                                                 long long row, const float* v) {
+  if (!p.fp8) {
+    uint8_t* base = (uint8_t*)(kv ? p.v[layer] : p.k[layer]) + row * 256;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      uint4 w;
+      w.x = pack_bf16(v[8 * c + 0], v[8 * c + 1]);
+      w.y = pack_bf16(v[8 * c + 2], v[8 * c + 3]);
+      w.z = pack_bf16(v[8 * c + 4], v[8 * c + 5]);
+      w.w = pack_bf16(v[8 * c + 6], v[8 * c + 7]);
+      *reinterpret_cast<uint4*>(base + 16 * c) = w;
+    }
+  } else {
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 128; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const float s = amax > 0.f ? amax / 448.f : 1.f;
+    uint8_t* base = (uint8_t*)(kv ? p.v[layer] : p.k[layer]) + row * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint32_t w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float* x = v + 16 * c + 4 * q;
+        const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+            make_float2(__fdiv_rn(x[0], s), __fdiv_rn(x[1], s)), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+            make_float2(__fdiv_rn(x[2], s), __fdiv_rn(x[3], s)), __NV_SATFINITE, __NV_E4M3);
+        w[q] = (uint32_t)lo | ((uint32_t)hi << 16);
+      }
+      *reinterpret_cast<uint4*>(base + 16 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    (kv ? p.v_scale[layer] : p.k_scale[layer])[row] = s;
+  }
+}
+
+__global__ void __launch_bounds__(kBrThreads, 1)
+    bridge_gemm_kernel(const __grid_constant__ CUtensorMap xmap,
+                       const __grid_constant__ CUtensorMap wmap, const BridgeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBrBarOff);
+  uint64_t* empty = full + kBrStages;
+  uint64_t* acc_full = empty + kBrStages;   // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long m_blocks = (p.T + kBrBM - 1) / kBrBM;
+  const long long n_tiles = m_blocks * p.n_layers;
+  const int k_blocks = p.hidden / kBrBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kBrStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&xmap);
+      tma_prefetch_desc(&wmap);
+      const uint64_t pol_x = policy_evict_first(), pol_w = policy_evict_last();
+      uint32_t it = 0;
+      bool ok = true;
+      for (long long tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        const long long mb = tile / p.n_layers;
+        const int layer = (int)(tile % p.n_layers);
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+          const int s = it % kBrStages;
+          const uint32_t ph = (it / kBrStages) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
+          uint8_t* a = smem + s * kBrStageBytes;
+          mbar_arrive_expect_tx(&full[s], kBrStageBytes);
+          tma_load_2d(a, &xmap, &full[s], kb * kBrBK, (int)(mb * kBrBM), pol_x);
+          tma_load_2d(a + kBrABytes, &wmap, &full[s], kb * kBrBK, layer * kBrBN, pol_w);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = bridge_idesc();
+      uint32_t it = 0, local = 0;
+      bool ok = true;
+      for (long long tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t use = local >> 1;
+        if (!mbar_wait(&acc_empty[acc], (use & 1) ^ 1)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kBrBN;
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+          const int s = it % kBrStages;
+          const uint32_t ph = (it / kBrStages) & 1;
+          if (!mbar_wait(&full[s], ph)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * kBrStageBytes);
+          const uint64_t adesc = sw128_kmajor_desc(a_addr);
+          const uint64_t bdesc = sw128_kmajor_desc(a_addr + kBrABytes);
+#pragma unroll
+          for (int k = 0; k < kBrBK / 16; ++k)  // +32 bytes along K per step
+            tc_mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
+          tc_commit(&empty[s]);
+        }
+        tc_commit(&acc_full[acc]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    uint32_t local = 0;
+    for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t use = local >> 1;
+      if (!mbar_wait(&acc_full[acc], use & 1)) break;
+      tc_fence_after();
+      const long long mb = tile / p.n_layers;
+      const int layer = (int)(tile % p.n_layers);
+      const long long tok = mb * kBrBM + quarter * 32 + lane;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kBrBN;
+#pragma unroll 1
+      for (int kv = 0; kv < 2; ++kv) {
+        float v[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(taddr + kv * 128 + c * 32, v + 32 * c);
+        tmem_ld_wait();
+        if (tok < p.T) bridge_store_row(p, layer, kv, p.row_offset + tok, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace hs2

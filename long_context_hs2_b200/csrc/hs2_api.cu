@@ -1,0 +1,357 @@
+// libhs2: C ABI of the hybrid-block hot path (see include/hs2.h).
+// One translation unit: every kernel header is included here.
+
+#include <hs2.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "bridge_gemm.cuh"
+#include "full_attn.cuh"
+#include "select.cuh"
+#include "sparse_attn.cuh"
+
+using namespace hs2;
+
+namespace {
+
+// ------------------------------------------------------------ TMA encode --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;  // resolved once; every thread resolves the same address
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D row-major tensor [rows][cols] of `elem`-byte elements, tile box
+// {box_cols, box_rows}, 128-byte swizzle.
+bool make_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, int elem,
+                 uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const CUtensorMapDataType dt =
+      elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)elem};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+bool aligned4(const void* p) { return ((uintptr_t)p & 3u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+hs2_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+}
+
+// ------------------------------------------------ full-attention plan --
+struct FullPlan {
+  int G, groups_per_seq, n_groups, n_splits, split_keys;
+  size_t off_part_o, off_part_ml, off_lse, off_hist, off_score, total;
+};
+
+bool check_attn_shape(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt) {
+  if (B < 1 || T < 1 || L < T || L > INT32_MAX || (int64_t)B * L > INT32_MAX) return false;
+  if (!(H == 8 || H == 16 || H == 32)) return false;
+  if (!(D == 64 || D == 128)) return false;
+  if (dt != HS2_KV_BF16 && dt != HS2_KV_FP8_E4M3) return false;
+  return true;
+}
+
+bool make_full_plan(int B, int T, int64_t L, int H, int D, int topk, int window, FullPlan* pl) {
+  (void)topk;
+  (void)window;
+  pl->G = kRows / H;
+  pl->groups_per_seq = (T + pl->G - 1) / pl->G;
+  pl->n_groups = B * pl->groups_per_seq;
+  const int64_t tiles = (L + kTile - 1) / kTile;
+  const int64_t target = 4LL * sm_count();
+  int64_t splits = (target + pl->n_groups - 1) / pl->n_groups;
+  splits = std::max<int64_t>(1, std::min<int64_t>(splits, tiles));
+  int64_t per = (L + splits - 1) / splits;
+  per = (per + kTile - 1) / kTile * kTile;
+  splits = (L + per - 1) / per;
+  pl->n_splits = (int)splits;
+  pl->split_keys = (int)per;
+  size_t off = 0;
+  pl->off_part_o = off;
+  off = align_up(off + (size_t)pl->n_groups * splits * kRows * D * 4, 256);
+  pl->off_part_ml = off;
+  off = align_up(off + (size_t)pl->n_groups * splits * kRows * 8, 256);
+  pl->off_lse = off;
+  off = align_up(off + (size_t)B * T * H * 4, 256);
+  pl->off_hist = off;
+  off = align_up(off + (size_t)B * T * kHistBins * 4, 256);
+  pl->off_score = off;
+  off = align_up(off + (size_t)B * T * (size_t)L * 4, 256);
+  pl->total = off;
+  return true;
+}
+
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+         cudaSuccess;
+}
+
+template <int D, bool FP8>
+hs2_status run_full(const CUtensorMap& km, const CUtensorMap& vm, const FullAttnParams& fp,
+                    const FullPlan& pl, const SelectParams& sp, cudaStream_t s) {
+  using SM = FullAttnSmem<D, FP8>;
+  auto kp = attn_partial_kernel<D, FP8>;
+  auto ks = attn_score_kernel<D, FP8>;
+  if (!set_smem(kp, SM::kBytes) || !set_smem(ks, SM::kScoreBytes)) return HS2_ERR_CUDA;
+  const int ctas = pl.n_groups * pl.n_splits;
+  kp<<<ctas, 160, SM::kBytes, s>>>(km, vm, fp);
+  if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+  const long long warps = (long long)pl.n_groups * kRows;
+  attn_combine_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(fp);
+  if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+  ks<<<ctas, 160, SM::kScoreBytes, s>>>(km, fp);
+  if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+  select_topk_kernel<<<(unsigned)(fp.B * fp.T), kSelThreads, 0, s>>>(sp);
+  return launch_status();
+}
+
+template <int MT, int D, bool FP8>
+hs2_status run_sparse(const SparseParams& p, cudaStream_t s) {
+  using SM = SparseSmem<MT, D, FP8>;
+  auto k = sparse_attn_kernel<MT, D, FP8>;
+  if (!set_smem(k, SM::kBytes)) return HS2_ERR_CUDA;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)((long long)p.B * p.T * p.cs));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = SM::kBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)p.cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k, p) != cudaSuccess) {
+    cudaGetLastError();
+    return HS2_ERR_CUDA;
+  }
+  return HS2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hs2_version(void) { return 100; }
+
+const char* hs2_status_string(hs2_status st) {
+  switch (st) {
+    case HS2_OK: return "ok";
+    case HS2_ERR_INVALID_ARG: return "invalid argument";
+    case HS2_ERR_UNSUPPORTED: return "unsupported shape or type";
+    case HS2_ERR_CUDA: return "CUDA error";
+    case HS2_ERR_WORKSPACE: return "workspace missing or too small";
+    case HS2_ERR_TIMEOUT: return "a kernel timed out waiting on a barrier";
+    case HS2_ERR_DEVICE: return "a kernel met an out-of-range index";
+  }
+  return "unknown status";
+}
+
+hs2_status hs2_last_device_status(hs2_stream_t stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return HS2_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return HS2_ERR_CUDA;
+  if (v && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return HS2_ERR_CUDA;
+  if (v & kStatusTimeout) return HS2_ERR_TIMEOUT;
+  if (v & kStatusBadIndex) return HS2_ERR_DEVICE;
+  return HS2_OK;
+}
+
+size_t hs2_full_attn_select_workspace(int B, int T, int64_t L, int H, int D, int topk,
+                                      int window, hs2_kv_dtype dt) {
+  if (!check_attn_shape(B, T, L, H, D, dt) || topk < 0 || window < 1 || topk + window > 4096)
+    return 0;
+  FullPlan pl;
+  make_full_plan(B, T, L, H, D, topk, window, &pl);
+  return pl.total;
+}
+
+hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, int T, int64_t L,
+                                int H, int D, float scale, int topk, int window,
+                                hs2_kv_dtype dt, float* O, float* lse, int32_t* idx,
+                                int32_t* n_sel, void* workspace, size_t workspace_bytes,
+                                hs2_stream_t stream) {
+  if (!Q || !kv || !kv->k || !kv->v || !O || !idx || !n_sel) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(kv->k) || !aligned16(kv->v) || !aligned16(O) ||
+      !aligned4(idx) || !aligned4(n_sel) || (lse && !aligned4(lse)))
+    return HS2_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || L < T || topk < 0 || window < 1 || !std::isfinite(scale))
+    return HS2_ERR_INVALID_ARG;
+  if (dt == HS2_KV_FP8_E4M3 && (!kv->k_scale || !kv->v_scale || !aligned4(kv->k_scale) ||
+                                !aligned4(kv->v_scale)))
+    return HS2_ERR_INVALID_ARG;
+  if (!check_attn_shape(B, T, L, H, D, dt) || topk + window > 4096) return HS2_ERR_UNSUPPORTED;
+  if (dt == HS2_KV_FP8_E4M3 && D != 128) return HS2_ERR_UNSUPPORTED;
+  FullPlan pl;
+  make_full_plan(B, T, L, H, D, topk, window, &pl);
+  if (!workspace || workspace_bytes < pl.total || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
+
+  const bool fp8 = dt == HS2_KV_FP8_E4M3;
+  const int elem = fp8 ? 1 : 2;
+  CUtensorMap km, vm;
+  const uint32_t box_cols = fp8 ? 128u : 64u;
+  if (!make_map_2d(&km, kv->k, (uint64_t)B * L, D, elem, box_cols, kTile) ||
+      !make_map_2d(&vm, kv->v, (uint64_t)B * L, D, elem, box_cols, kTile))
+    return HS2_ERR_CUDA;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  FullAttnParams fp;
+  fp.q = static_cast<const __nv_bfloat16*>(Q);
+  fp.k_scale = fp8 ? kv->k_scale : nullptr;
+  fp.v_scale = fp8 ? kv->v_scale : nullptr;
+  fp.part_o = reinterpret_cast<float*>(ws + pl.off_part_o);
+  fp.part_ml = reinterpret_cast<float2*>(ws + pl.off_part_ml);
+  fp.lse = reinterpret_cast<float*>(ws + pl.off_lse);
+  fp.lse_out = lse;
+  fp.o = O;
+  fp.score = reinterpret_cast<float*>(ws + pl.off_score);
+  fp.hist = reinterpret_cast<unsigned*>(ws + pl.off_hist);
+  fp.B = B;
+  fp.T = T;
+  fp.H = H;
+  fp.D = D;
+  fp.L = L;
+  fp.G = pl.G;
+  fp.groups_per_seq = pl.groups_per_seq;
+  fp.n_splits = pl.n_splits;
+  fp.split_keys = pl.split_keys;
+  fp.window = window;
+  fp.scale_log2 = scale * kLog2e;
+
+  SelectParams sp;
+  sp.score = fp.score;
+  sp.hist = fp.hist;
+  sp.idx = idx;
+  sp.n_sel = n_sel;
+  sp.T = T;
+  sp.L = L;
+  sp.topk = topk;
+  sp.window = window;
+  sp.slots = topk + window;
+
+  cudaStream_t s = (cudaStream_t)stream;
+  if (fp8) return run_full<128, true>(km, vm, fp, pl, sp, s);
+  if (D == 128) return run_full<128, false>(km, vm, fp, pl, sp, s);
+  return run_full<64, false>(km, vm, fp, pl, sp, s);
+}
+
+hs2_status hs2_sparse_attn(const void* Q, const hs2_kv_cache* kv, int B, int T, int64_t L, int H,
+                           int D, float scale, const int32_t* idx, const int32_t* n_sel,
+                           int slots, hs2_kv_dtype dt, float* O, hs2_stream_t stream) {
+  if (!Q || !kv || !kv->k || !kv->v || !idx || !n_sel || !O) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(kv->k) || !aligned16(kv->v) || !aligned16(O) ||
+      !aligned4(idx) || !aligned4(n_sel))
+    return HS2_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || L < T || slots < 1 || !std::isfinite(scale)) return HS2_ERR_INVALID_ARG;
+  if (dt == HS2_KV_FP8_E4M3 && (!kv->k_scale || !kv->v_scale || !aligned4(kv->k_scale) ||
+                                !aligned4(kv->v_scale)))
+    return HS2_ERR_INVALID_ARG;
+  if (!check_attn_shape(B, T, L, H, D, dt) || slots > 4096) return HS2_ERR_UNSUPPORTED;
+  if (dt == HS2_KV_FP8_E4M3 && D != 128) return HS2_ERR_UNSUPPORTED;
+
+  SparseParams p;
+  p.q = static_cast<const __nv_bfloat16*>(Q);
+  p.k = static_cast<const uint8_t*>(kv->k);
+  p.v = static_cast<const uint8_t*>(kv->v);
+  p.k_scale = kv->k_scale;
+  p.v_scale = kv->v_scale;
+  p.idx = idx;
+  p.n_sel = n_sel;
+  p.o = O;
+  p.B = B;
+  p.T = T;
+  p.H = H;
+  p.D = D;
+  p.slots = slots;
+  p.L = L;
+  p.scale_log2 = scale * kLog2e;
+  const long long queries = (long long)B * T;
+  const int sms = sm_count();
+  int cs = 1;
+  while (cs < 8 && queries * cs * 2 <= sms && cs * kSpTile < slots) cs *= 2;
+  p.cs = cs;
+  const bool fp8 = dt == HS2_KV_FP8_E4M3;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (fp8) return H == 32 ? run_sparse<2, 128, true>(p, s) : run_sparse<1, 128, true>(p, s);
+  if (D == 128) return H == 32 ? run_sparse<2, 128, false>(p, s) : run_sparse<1, 128, false>(p, s);
+  return H == 32 ? run_sparse<2, 64, false>(p, s) : run_sparse<1, 64, false>(p, s);
+}
+
+}  // extern "C"
+
+extern "C" hs2_status hs2_bridge_kv(const void* X, int64_t T, int hidden, const void* Wt,
+                                    int n_layers, int D, hs2_kv_dtype out_dtype,
+                                    const hs2_kv_cache* caches, int64_t cache_row_offset,
+                                    hs2_stream_t stream) {
+  if (!X || !Wt || !caches || T < 1 || hidden < 1 || n_layers < 1 || cache_row_offset < 0)
+    return HS2_ERR_INVALID_ARG;
+  if (out_dtype != HS2_KV_BF16 && out_dtype != HS2_KV_FP8_E4M3) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Wt)) return HS2_ERR_INVALID_ARG;
+  const bool fp8 = out_dtype == HS2_KV_FP8_E4M3;
+  for (int l = 0; l < n_layers; ++l) {
+    const hs2_kv_cache& c = caches[l];
+    if (!c.k || !c.v || !aligned16(c.k) || !aligned16(c.v)) return HS2_ERR_INVALID_ARG;
+    if (fp8 && (!c.k_scale || !c.v_scale || !aligned4(c.k_scale) || !aligned4(c.v_scale)))
+      return HS2_ERR_INVALID_ARG;
+  }
+  if (D != 128 || hidden % kBrBK != 0 || n_layers > kBrMaxLayers || T > INT32_MAX - kBrBM)
+    return HS2_ERR_UNSUPPORTED;
+  CUtensorMap xm, wm;
+  if (!make_map_2d(&xm, X, (uint64_t)T, (uint64_t)hidden, 2, kBrBK, kBrBM) ||
+      !make_map_2d(&wm, Wt, (uint64_t)n_layers * kBrBN, (uint64_t)hidden, 2, kBrBK, kBrBN))
+    return HS2_ERR_CUDA;
+  BridgeParams p;
+  std::memset(&p, 0, sizeof(p));
+  for (int l = 0; l < n_layers; ++l) {
+    p.k[l] = caches[l].k;
+    p.v[l] = caches[l].v;
+    p.k_scale[l] = fp8 ? caches[l].k_scale : nullptr;
+    p.v_scale[l] = fp8 ? caches[l].v_scale : nullptr;
+  }
+  p.T = T;
+  p.row_offset = cache_row_offset;
+  p.hidden = hidden;
+  p.n_layers = n_layers;
+  p.fp8 = fp8 ? 1 : 0;
+  if (!set_smem(bridge_gemm_kernel, kBrSmemBytes)) return HS2_ERR_CUDA;
+  const long long tiles = (T + kBrBM - 1) / kBrBM * n_layers;
+  const int grid = (int)std::min<long long>(tiles, sm_count());
+  bridge_gemm_kernel<<<grid, kBrThreads, kBrSmemBytes, (cudaStream_t)stream>>>(xm, wm, p);
+  return launch_status();
+}

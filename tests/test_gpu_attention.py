@@ -1,0 +1,138 @@
+"""GPU parity: hs2_full_attn_select and hs2_sparse_attn against the CPU oracle.
+
+Every case runs the CUDA path through the C ABI and the oracle on the same
+seeded input bytes.  O and O' must be within the stated max-abs tolerance
+(1e-2 bf16 cache, 3e-2 E4M3 cache); selected sets must match except for
+swaps among candidates whose oracle score lies within 1e-3 (relative) of the
+k-th score; the forced window and the planted needles must be selected.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import hs2_testlib as tl
+from hs2_synth import WORKLOADS, make_attention_inputs
+import long_context_hs2_b200 as hs2
+
+pytestmark = pytest.mark.gpu
+
+
+def _positions(wl, rows):
+    return [wl.L - wl.T + (r % wl.T) for r in rows]
+
+
+def _check_block(wl, rows=None, sparse_layers=None, needles=True):
+    inp = make_attention_inputs(wl, needles=needles)
+    di = tl.DeviceInputs(inp)
+    g = tl.run_full(di)
+    rows = np.arange(wl.B * wl.T) if rows is None else np.asarray(rows)
+    orc = tl.oracle_full(inp, rows=rows)
+    tol = tl.TOL_FP8 if di.fp8 else tl.TOL_BF16
+    assert tl.max_abs(g["o"][rows], orc["o"]) <= tol
+    assert tl.max_abs(g["lse"][rows], orc["lse"]) <= 1e-3
+    differ = tl.check_selection(g["idx"][rows], g["n_sel"][rows], orc, _positions(wl, rows),
+                                wl.topk, wl.window)
+    assert differ <= max(1, len(rows) // 50)
+    sel_rows = {int(r): k for k, r in enumerate(rows)}
+    for b, j, t in inp.needles:
+        r = int(b) * wl.T + int(t)
+        if r in sel_rows:
+            assert j in g["idx"][r, : g["n_sel"][r]], ("needle not selected", b, j, t)
+    layers = range(wl.n_sparse) if sparse_layers is None else sparse_layers
+    slots = wl.topk + wl.window
+    # each sparse layer reuses the oracle's indices: isolates the sparse kernel
+    full_idx = np.full((wl.B * wl.T, slots), -1, dtype=np.int32)
+    full_ns = np.zeros(wl.B * wl.T, dtype=np.int32)
+    full_idx[rows] = orc["idx"]
+    full_ns[rows] = orc["n_sel"]
+    for layer in layers:
+        o_gpu = tl.run_sparse(di, layer, full_idx, full_ns, slots)
+        o_orc = tl.oracle_sparse(inp, layer, full_idx, full_ns, rows=rows)
+        assert tl.max_abs(o_gpu[rows], o_orc) <= tol
+    # the GPU's own indices, end to end, on rows whose sets equal the oracle's
+    same = [k for k, r in enumerate(rows)
+            if np.array_equal(g["idx"][r], orc["idx"][k])]
+    if layers and same:
+        layer = list(layers)[0]
+        o_gpu = tl.run_sparse(di, layer, g["idx_dev"], g["nsel_dev"], slots)
+        o_orc = tl.oracle_sparse(inp, layer, full_idx, full_ns, rows=rows[same])
+        assert tl.max_abs(o_gpu[rows[same]], o_orc) <= tol
+    return g
+
+
+def test_tiny_block():
+    _check_block(WORKLOADS["tiny"])
+
+
+def test_decode_bf16_ragged():
+    _check_block(WORKLOADS["decode_bf16_32k"].resized(B=3, L=5003, n_needles=12))
+
+
+def test_decode_bf16_32k():
+    _check_block(WORKLOADS["decode_bf16_32k"])
+
+
+def test_decode_fp8_ragged():
+    _check_block(WORKLOADS["decode_fp8_256k"].resized(B=2, L=9007, n_needles=20))
+
+
+def test_decode_fp8_256k():
+    _check_block(WORKLOADS["decode_fp8_256k"])
+
+
+def test_chunk_fp8_small():
+    wl = WORKLOADS["chunk_fp8_1m"].resized(T=200, L=20011, n_needles=40, n_sparse=1)
+    rows = np.unique(np.r_[0, 199, np.random.default_rng(1).integers(0, 200, 30)])
+    _check_block(wl, rows=rows)
+
+
+def test_chunk_bf16_heads8_d64():
+    wl = WORKLOADS["tiny"].resized(T=300, L=3001, n_needles=10)
+    _check_block(wl)
+
+
+def test_heads16_bf16():
+    wl = WORKLOADS["decode_bf16_32k"].resized(B=2, T=3, L=4000, H=16, n_needles=6)
+    _check_block(wl)
+
+
+def test_context_within_budget_sparse_equals_dense():
+    # every position is selected, so a sparse layer with the full layer's own
+    # queries must reproduce the full layer's output
+    wl = WORKLOADS["decode_bf16_32k"].resized(B=2, T=5, L=1100, n_needles=0, n_sparse=1)
+    inp = make_attention_inputs(wl, needles=False)
+    inp.q_sparse[0] = inp.q
+    di = tl.DeviceInputs(inp)
+    g = tl.run_full(di)
+    assert (g["n_sel"] == np.tile(wl.L - wl.T + np.arange(wl.T) + 1, wl.B)).all()
+    o2 = tl.run_sparse(di, 0, g["idx_dev"], g["nsel_dev"], wl.topk + wl.window)
+    assert tl.max_abs(o2, g["o"]) <= 2e-3
+
+
+def test_short_context_and_zero_topk():
+    wl = WORKLOADS["tiny"].resized(T=50, L=50, n_needles=0, topk=16, window=128)
+    _check_block(wl, needles=False)
+    wl = WORKLOADS["tiny"].resized(T=40, L=700, n_needles=0, topk=0, window=32)
+    _check_block(wl, needles=False)
+
+
+def test_sparse_empty_selection_gives_zero():
+    wl = WORKLOADS["decode_bf16_32k"].resized(B=2, L=512, n_needles=0, n_sparse=1)
+    di = tl.DeviceInputs(make_attention_inputs(wl, needles=False))
+    idx = -np.ones((2, 16), dtype=np.int32)
+    o = tl.run_sparse(di, 0, idx, np.zeros(2, dtype=np.int32), 16)
+    assert np.all(o == 0)
+
+
+def test_sparse_out_of_range_index_is_reported():
+    wl = WORKLOADS["decode_bf16_32k"].resized(B=1, L=512, n_needles=0, n_sparse=1)
+    di = tl.DeviceInputs(make_attention_inputs(wl, needles=False))
+    idx = np.arange(16, dtype=np.int32)[None, :].copy()
+    idx[0, 5] = 512 + 40   # past the cache: the kernel must skip it and report
+    nsel = np.array([16], dtype=np.int32)
+    O = torch.empty(1, 1, wl.H, wl.D, dtype=torch.float32, device="cuda")
+    hs2.hs2_sparse_attn(di.q_sparse[0], di.kv, 1, 1, wl.L, wl.H, wl.D, wl.scale, tl.dev(idx),
+                        tl.dev(nsel), 16, di.dt, O)
+    assert hs2.hs2_last_device_status() == 6
+    assert hs2.hs2_last_device_status() == 0   # cleared by the read
