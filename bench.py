@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Benchmark of the HySparse2 hybrid-block hot path on B200.
+
+One step = one hybrid block on the decode workload (8 sequences x 1 new query
+at 32,768 tokens of bf16 MQA cache, 32 query heads, head_dim 128): the
+full-attention layer with top-1024 + recent-128 selection, then three
+sparse-attention layers that reuse its KV cache and indices, each with its
+own queries.  The metric is hybrid-block decode tokens/s (queries through the
+whole block per second).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hs2|reference]
+
+N > 1 runs one process per GPU under torch.distributed.run: every rank runs
+its own replica of the workload (weak scaling; the decode path shards by
+sequence with no exchange), times are the max over ranks.  --impl reference
+times the CPU oracle on the same workload (rank 0 only).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hs2_synth import WORKLOADS, make_attention_inputs  # noqa: E402
+
+WORKLOAD = "decode_bf16_32k"
+L2_FLUSH_BYTES = 512 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["hs2", "reference"], default="hs2")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------------- oracle arm --
+def oracle_rows_per_s(inp, rows, n_sparse):
+    """Oracle time for the block on `rows` query rows (full + select + sparse layers)."""
+    import oracle
+    wl = inp.wl
+    t0 = time.perf_counter()
+    r = oracle.full_attn_select(inp.q, inp.k, inp.v, inp.k_scale, inp.v_scale, scale=wl.scale,
+                                topk=wl.topk, window=wl.window, rows=rows)
+    idx = np.full((wl.B * wl.T, wl.topk + wl.window), -1, dtype=np.int32)
+    ns = np.zeros(wl.B * wl.T, dtype=np.int32)
+    idx[rows] = r["idx"]
+    ns[rows] = r["n_sel"]
+    for layer in range(n_sparse):
+        oracle.sparse_attn(inp.q_sparse[layer], inp.k, inp.v, inp.k_scale, inp.v_scale, idx, ns,
+                           scale=wl.scale, rows=rows)
+    dt = time.perf_counter() - t0
+    return len(rows) / dt, dt, oracle.threads()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    wl = WORKLOADS[WORKLOAD]
+    inp = make_attention_inputs(wl)
+    rows = np.arange(1)          # one sequence's query per step: a bounded sample
+    for _ in range(args.warmup):
+        oracle_rows_per_s(inp, rows, wl.n_sparse)
+    times = []
+    cores = 1
+    for s in range(args.steps):
+        rows = np.array([s % (wl.B * wl.T)])
+        _, dt, cores = oracle_rows_per_s(inp, rows, wl.n_sparse)
+        times.append(dt)
+    ms = 1000.0 * sum(times) / len(times)
+    value = 1000.0 / ms
+    line = {
+        "impl": "reference", "metric": "hybrid-block decode tokens/s", "value": value,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": wl.B, "T": wl.T, "L": wl.L, "H": wl.H, "D": wl.D,
+                   "kv": wl.kv_dtype, "topk": wl.topk, "window": wl.window,
+                   "sparse_layers": wl.n_sparse},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "1 of the 8 sequences per step (full attention + selection "
+                                   "+ 3 sparse layers), plain C++ fp64 oracle"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm --
+def run_hs2(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+    import long_context_hs2_b200 as hs2
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    hs2.load_library()
+    base = WORKLOADS[WORKLOAD]
+    wl = base.resized(seed=base.seed + 1000 * rank)       # each rank: its own sequences
+    inp = make_attention_inputs(wl)
+    B, T, L, H, D = wl.B, wl.T, wl.L, wl.H, wl.D
+    slots = wl.topk + wl.window
+    dt = hs2.HS2_KV_BF16
+
+    def up(a, dtype):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(dtype)
+
+    k = up(inp.k, torch.bfloat16)
+    v = up(inp.v, torch.bfloat16)
+    kv = hs2.kv_cache(k, v)
+    qs = [up(q, torch.bfloat16) for q in [inp.q] + inp.q_sparse]
+    ws_bytes = hs2.hs2_full_attn_select_workspace(B, T, L, H, D, wl.topk, wl.window, dt)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    outs = [torch.empty(B, T, H, D, dtype=torch.float32, device="cuda") for _ in qs]
+    idx = torch.empty(B, T, slots, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(B, T, dtype=torch.int32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(q_list):
+        hs2.hs2_full_attn_select(q_list[0], kv, B, T, L, H, D, wl.scale, wl.topk, wl.window, dt,
+                                 outs[0], None, idx, nsel, ws, ws_bytes, stream)
+        for s in range(wl.n_sparse):
+            hs2.hs2_sparse_attn(q_list[1 + s], kv, B, T, L, H, D, wl.scale, idx, nsel, slots, dt,
+                                outs[1 + s], stream)
+
+    def full_layer(q_list):
+        hs2.hs2_full_attn_select(q_list[0], kv, B, T, L, H, D, wl.scale, wl.topk, wl.window, dt,
+                                 outs[0], None, idx, nsel, ws, ws_bytes)
+
+    def sparse_layers(q_list):
+        for s in range(wl.n_sparse):
+            hs2.hs2_sparse_attn(q_list[1 + s], kv, B, T, L, H, D, wl.scale, idx, nsel, slots, dt,
+                                outs[1 + s])
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(qs)
+    torch.cuda.synchronize()
+    st = hs2.hs2_last_device_status()
+    if st != 0:
+        raise RuntimeError("device status after warm-up: " + hs2.hs2_status_string(st))
+
+    # The block's launches are captured once into CUDA graphs (full layer; the
+    # three sparse layers) and replayed every step, as a decode loop would.
+    d_q = [torch.empty_like(q) for q in qs]
+    for dq, q in zip(d_q, qs):
+        dq.copy_(q)
+    g_full, g_sparse = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_full):
+        full_layer(d_q)
+    with torch.cuda.graph(g_sparse):
+        sparse_layers(d_q)
+    for _ in range(args.warmup):
+        flush.zero_()
+        g_full.replay()
+        g_sparse.replay()
+    torch.cuda.synchronize()
+
+    # ---- device-timed steps (inputs resident in HBM; L2 flushed before each)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local if world == 1 else int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        g_full.replay()
+        e1.record(stream)
+        g_sparse.replay()
+        e2.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    full_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    sparse_ms = [b.elapsed_time(c) / wl.n_sparse for _, b, c in ev]
+    st = hs2.hs2_last_device_status()
+    if st != 0:
+        raise RuntimeError("device status after timing: " + hs2.hs2_status_string(st))
+
+    # ---- end to end: pinned host queries in, outputs back, every step
+    h_q = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for q in qs]
+    for hq, q in zip(h_q, qs):
+        hq.copy_(q.cpu())
+    h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h_idx = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
+    h_ns = torch.empty(nsel.shape, dtype=nsel.dtype, pin_memory=True)
+    h2d = sum(q.numel() * q.element_size() for q in qs)
+    d2h = sum(o.numel() * o.element_size() for o in outs) + idx.numel() * 4 + nsel.numel() * 4
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        a, c = e2e_ev[i]
+        a.record(stream)
+        for dq, hq in zip(d_q, h_q):
+            dq.copy_(hq, non_blocking=True)
+        g_full.replay()
+        g_sparse.replay()
+        for ho, o in zip(h_out, outs):
+            ho.copy_(o, non_blocking=True)
+        h_idx.copy_(idx, non_blocking=True)
+        h_ns.copy_(nsel, non_blocking=True)
+        c.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = [a.elapsed_time(c) for a, c in e2e_ev]
+
+    def agg(xs):
+        m = float(np.mean(xs))
+        if world > 1:
+            t = torch.tensor([m], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            m = float(t.item())
+        return m
+
+    ms = agg(step_ms)
+    full = agg(full_ms)
+    sparse = agg(sparse_ms)
+    e2e = agg(e2e_ms)
+    peak, peak_kind = measured_peaks()
+    kv_bytes = 2 * B * L * D * 2
+    full_bytes = kv_bytes + B * T * H * D * 2 + B * T * H * D * 4 + B * T * slots * 4 + B * T * 4
+    sparse_bytes = B * T * slots * 2 * D * 2 + B * T * H * D * 2 + B * T * H * D * 4 + B * T * slots * 4
+    achieved = full_bytes / (full * 1e-3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic_full_attn_select_decode_bf16_32k.json")
+    if os.path.exists(tpath):
+        try:
+            with open(tpath) as f:
+                traffic = json.load(f).get("bytes_per_launch")
+        except Exception:
+            traffic = None
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rps, dts, cores = oracle_rows_per_s(inp, np.arange(B * T), wl.n_sparse)
+        cpu = {"value": rps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": "one full step: %d sequences x 1 query, full attention + selection + "
+                         "%d sparse layers (%.1f s)" % (B, wl.n_sparse, dts)}
+    del g_full, g_sparse
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    tokens = B * T * world
+    line = {
+        "metric": "hybrid-block decode tokens/s",
+        "value": tokens / (ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "T": T, "L": L, "H": H, "D": D,
+                   "kv": "bf16", "topk": wl.topk, "window": wl.window,
+                   "sparse_layers": wl.n_sparse, "parallelism": "replicas (dp%d)" % world,
+                   "l2": "flushed before each step (512 MB write)"},
+        "e2e": {"value": tokens / (e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": (4 + wl.n_sparse) * args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "hs2_full_attn_select (attn_partial, attn_combine, attn_score, "
+                               "select_topk)", "peak_source": peak_kind},
+        "sparse_layer": {"ms": sparse, "achieved_gbs": sparse_bytes / (sparse * 1e-3) / 1e9,
+                         "frac": sparse_bytes / (sparse * 1e-3) / 1e9 / peak},
+        "full_ms": full,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_hs2(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -6,12 +6,13 @@
 // split of that group's causal key range.  Warps 0-3 each take 16 keys of
 // every 64-key tile; warp 4 issues the TMA loads of the tile ring.
 //   attn_partial : per (group, split) the base-2 running max m, sum l and the
-//                  un-normalised O of the split (flash-decoding partials).
-//   attn_combine : merges the splits into O and lse (natural log), and clears
-//                  the per-query level-1 histograms of the selection.
-//   attn_score   : second pass over K (L2-resident when it fits): for every
-//                  candidate j <= i - window, score_j = sum_h exp(s_hj - lse_h),
-//                  written as fp32, plus a histogram of the score's top bits.
+//                  un-normalised O of the split (flash-decoding partials); the
+//                  group's first split also clears its level-1 histograms.
+//   attn_score   : merges the splits into lse (every CTA, for its group) and O
+//                  (each row by one CTA of the group), then makes a second pass
+//                  over K (L2-resident when it fits): for every candidate
+//                  j <= i - window, score_j = sum_h exp(s_hj - lse_h), written as
+//                  fp32, plus a histogram of the score's top bits.
 #pragma once
 
 #include "attn_warp.cuh"
@@ -38,6 +39,7 @@ struct FullAttnParams {
   int B, T, H, D;
   long long L;
   int G, groups_per_seq, n_splits, split_keys, window;
+  int score_splits, score_keys;  // split of the score pass (finer than the partials')
   float scale_log2;
 };
 
@@ -62,7 +64,8 @@ struct FullAttnSmem {
   static constexpr int kScoreStages = 4;
   static constexpr int kScoreHistOff = kScoreStages * kScoreStageBytes + kScoreStagingBytes;
   static constexpr int kScoreQOff = kScoreHistOff + 4 * kHistBins * 4;
-  static constexpr int kScoreBarOff = kScoreQOff + kQBytes;
+  static constexpr int kScoreLseOff = kScoreQOff + kQBytes;
+  static constexpr int kScoreBarOff = kScoreLseOff + kRows * 4;
   static constexpr int kScoreBytes = kScoreBarOff + 2 * kScoreStages * 8 + 1024;
 };
 
@@ -124,6 +127,12 @@ __global__ void __launch_bounds__(160) attn_partial_kernel(const __grid_constant
   const long long k_hi = min(k_lo + p.split_keys, i_last + 1);
   const long long part = (long long)grp * p.n_splits + split;
 
+  if (split == 0) {  // clear the group's level-1 selection histograms
+    for (int u = threadIdx.x; u < p.G * kHistBins; u += blockDim.x) {
+      const int t = t0 + u / kHistBins;
+      if (t < p.T) p.hist[((long long)b * p.T + t) * kHistBins + (u % kHistBins)] = 0u;
+    }
+  }
   if (k_lo >= k_hi) {  // empty split: neutral partial
     for (int u = threadIdx.x; u < kRows * D; u += blockDim.x) p.part_o[part * kRows * D + u] = 0.f;
     if (threadIdx.x < kRows) p.part_ml[part * kRows + threadIdx.x] = make_float2(kNegInf, 0.f);
@@ -277,54 +286,7 @@ __global__ void __launch_bounds__(160) attn_partial_kernel(const __grid_constant
   }
 }
 
-// One warp per (group, row): merges the splits, writes O and lse.  All
-// threads also clear the level-1 selection histograms.
-template <int D>
-__global__ void __launch_bounds__(256) attn_combine_kernel(const FullAttnParams p) {
-  const long long n_hist = (long long)p.B * p.T * kHistBins;
-  for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < n_hist;
-       u += (long long)gridDim.x * blockDim.x)
-    p.hist[u] = 0u;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long wid = (long long)blockIdx.x * 8 + warp;
-  const long long groups = (long long)p.B * p.groups_per_seq;
-  if (wid >= groups * kRows) return;
-  const int r = (int)(wid % kRows);
-  const long long grp = wid / kRows;
-  const int b = (int)(grp / p.groups_per_seq);
-  const int t = (int)(grp % p.groups_per_seq) * p.G + r / p.H;
-  const int h = r % p.H;
-  if (t >= p.T) return;
-  float M = kNegInf;
-  for (int s = 0; s < p.n_splits; ++s) M = fmaxf(M, p.part_ml[(grp * p.n_splits + s) * kRows + r].x);
-  float lt = 0.f;
-  float acc[D / 32];
-#pragma unroll
-  for (int k = 0; k < D / 32; ++k) acc[k] = 0.f;
-  if (M != kNegInf) {
-    for (int s = 0; s < p.n_splits; ++s) {
-      const long long part = grp * p.n_splits + s;
-      const float2 v = p.part_ml[part * kRows + r];
-      const float fct = (v.x == kNegInf) ? 0.f : fast_exp2(v.x - M);
-      lt += v.y * fct;
-      const float* po = p.part_o + (part * kRows + r) * D;
-#pragma unroll
-      for (int k = 0; k < D / 32; ++k) acc[k] += fct * po[lane + 32 * k];
-    }
-  }
-  const float inv = lt > 0.f ? 1.f / lt : 0.f;
-  float* out = p.o + (((long long)b * p.T + t) * p.H + h) * D;
-#pragma unroll
-  for (int k = 0; k < D / 32; ++k) out[lane + 32 * k] = acc[k] * inv;
-  if (lane == 0) {
-    const float lse = (M + log2f(lt)) * 0.69314718055994531f;
-    const long long li = ((long long)b * p.T + t) * p.H + h;
-    p.lse[li] = lse;
-    if (p.lse_out) p.lse_out[li] = lse;
-  }
-}
-
-template <int D, bool FP8>
+template <int D, bool FP8, int G>
 __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__ CUtensorMap kmap,
                                                          const FullAttnParams p) {
   using SM = FullAttnSmem<D, FP8>;
@@ -336,17 +298,63 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kScoreBarOff);
   uint64_t* empty = full + kStages;
 
-  const int split = blockIdx.x % p.n_splits;
-  const int grp = blockIdx.x / p.n_splits;
+  const int split = blockIdx.x % p.score_splits;
+  const int grp = blockIdx.x / p.score_splits;
   const int b = grp / p.groups_per_seq;
-  const int t0 = (grp % p.groups_per_seq) * p.G;
-  const int t_last = min(p.T, t0 + p.G) - 1;
+  const int t0 = (grp % p.groups_per_seq) * G;
+  const int t_last = min(p.T, t0 + G) - 1;
   const long long i_last = p.L - p.T + t_last;
-  const long long k_lo = (long long)split * p.split_keys;
-  const long long k_hi = min(k_lo + p.split_keys, i_last - p.window + 1);
+  const long long k_lo = (long long)split * p.score_keys;
+  const long long k_hi = min(k_lo + p.score_keys, i_last - p.window + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* lse2_s = reinterpret_cast<float*>(smem + SM::kScoreLseOff);
+
+  // ---- merge of the splits: lse of the group's rows (base 2) in every CTA;
+  //      O of row r in the CTA whose score-split index is r mod score_splits.
+  if (warp < kConsumers) {
+    for (int r = warp; r < kRows; r += kConsumers) {
+      const int t = t0 + r / p.H;
+      const float2* ml = p.part_ml + (long long)grp * p.n_splits * kRows + r;
+      float M = kNegInf;
+      for (int sp = lane; sp < p.n_splits; sp += 32) M = fmaxf(M, ml[(long long)sp * kRows].x);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      float lt = 0.f;
+      if (M != kNegInf)
+        for (int sp = lane; sp < p.n_splits; sp += 32) {
+          const float2 v = ml[(long long)sp * kRows];
+          lt += v.x == kNegInf ? 0.f : v.y * fast_exp2(v.x - M);
+        }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
+      const float l2 = M + log2f(lt);
+      if (lane == 0) lse2_s[r] = l2;
+      if (t < p.T && (r % p.score_splits) == split) {
+        const long long li = ((long long)b * p.T + t) * p.H + r % p.H;
+        if (lane == 0) {
+          p.lse[li] = l2 * 0.69314718055994531f;
+          if (p.lse_out) p.lse_out[li] = l2 * 0.69314718055994531f;
+        }
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        float acc[D / 32];
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) acc[k] = 0.f;
+        const float* po = p.part_o + ((long long)grp * p.n_splits * kRows + r) * D;
+#pragma unroll 4
+        for (int sp = 0; sp < p.n_splits; ++sp) {
+          const float2 v = ml[(long long)sp * kRows];
+          const float f = (v.x == kNegInf) ? 0.f : fast_exp2(v.x - M) * inv;
+#pragma unroll
+          for (int k = 0; k < D / 32; ++k) acc[k] += f * po[(long long)sp * kRows * D + lane + 32 * k];
+        }
+        float* out = p.o + li * D;
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) out[lane + 32 * k] = acc[k];
+      }
+    }
+  }
   if (k_lo >= k_hi) return;
   const int n_tiles = (int)((k_hi - k_lo + kTile - 1) / kTile);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
   }
 
   load_q_tile<D>(p, b, t0, qs);
-  for (int u = threadIdx.x; u < p.G * kHistBins; u += kConsumers * 32) hist_s[u] = 0u;
+  for (int u = threadIdx.x; u < G * kHistBins; u += kConsumers * 32) hist_s[u] = 0u;
   consumer_sync();
 
   const int g = lane >> 2, c = lane & 3;
@@ -389,7 +397,7 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
       const int t = t0 + tl;
       qry[mt][h] = tl;
       i_row[mt][h] = (t < p.T) ? p.L - p.T + t : -1;  // -1: no candidates
-      lse2[mt][h] = (t < p.T) ? p.lse[((long long)b * p.T + t) * p.H + r % p.H] * kLog2e : 0.f;
+      lse2[mt][h] = (t < p.T) ? lse2_s[r] : 0.f;
     }
   const float* ksc = FP8 ? p.k_scale + (long long)b * p.L : nullptr;
   const uint32_t q_base = smem_u32(qs);
@@ -420,10 +428,11 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
-    // acc[tl][nt][j]: head-sum of query tl for key nt*8 + 2c + j
-    float acc[4][2][2];
+    // acc[tl][nt][j]: head-sum of query tl (rows tl*H .. tl*H+H-1) for key nt*8 + 2c + j.
+    // Thread rows are mt*16 + g + 8h, so query tl = (mt*16 + 8h + g) / H.
+    float acc[G][2][2];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+    for (int q = 0; q < G; ++q)
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) acc[q][nt][0] = acc[q][nt][1] = 0.f;
 #pragma unroll
@@ -438,13 +447,21 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
           for (int h = 0; h < 2; ++h) {
             const bool ok = key <= i_row[mt][h] - p.window;
             const float pr = ok ? fast_exp2(x[mt][nt][2 * h + j] * (p.scale_log2 * ks) - lse2[mt][h]) : 0.f;
+            if (G == 1) {
+              acc[0][nt][j] += pr;
+            } else {
+              // rows of this thread: mt*16 + 8h + g; with H = 32/G, query = row / H
+              constexpr int kH = 32 / G;
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (q == qry[mt][h]) acc[q][nt][j] += pr;
+              for (int q = 0; q < G; ++q)
+                if (((mt * 16 + 8 * h) / kH == q && kH >= 16) ||
+                    (kH == 8 && (mt * 16 + 8 * h) / 8 == q))
+                  acc[q][nt][j] += pr;
+            }
           }
       }
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+    for (int q = 0; q < G; ++q)
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -457,8 +474,7 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
         }
     if (g == 0) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (q >= p.G) break;
+      for (int q = 0; q < G; ++q) {
         const int t = t0 + q;
         if (t >= p.T) break;
         const long long i_q = p.L - p.T + t;
@@ -478,7 +494,7 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
     }
   }
   consumer_sync();
-  for (int u = threadIdx.x; u < p.G * kHistBins; u += kConsumers * 32) {
+  for (int u = threadIdx.x; u < G * kHistBins; u += kConsumers * 32) {
     const unsigned cnt = hist_s[u];
     const int q = u / kHistBins;
     const int t = t0 + q;

@@ -72,7 +72,7 @@ hs2_status launch_status() {
 
 // ------------------------------------------------ full-attention plan --
 struct FullPlan {
-  int G, groups_per_seq, n_groups, n_splits, split_keys;
+  int G, groups_per_seq, n_groups, n_splits, split_keys, score_splits, score_keys;
   size_t off_part_o, off_part_ml, off_lse, off_hist, off_score, total;
 };
 
@@ -91,7 +91,7 @@ bool make_full_plan(int B, int T, int64_t L, int H, int D, int topk, int window,
   pl->groups_per_seq = (T + pl->G - 1) / pl->G;
   pl->n_groups = B * pl->groups_per_seq;
   const int64_t tiles = (L + kTile - 1) / kTile;
-  const int64_t target = 4LL * sm_count();
+  const int64_t target = sm_count();  // about one wave of CTAs
   int64_t splits = (target + pl->n_groups - 1) / pl->n_groups;
   splits = std::max<int64_t>(1, std::min<int64_t>(splits, tiles));
   int64_t per = (L + splits - 1) / splits;
@@ -99,6 +99,13 @@ bool make_full_plan(int B, int T, int64_t L, int H, int D, int topk, int window,
   splits = (L + per - 1) / per;
   pl->n_splits = (int)splits;
   pl->split_keys = (int)per;
+  // the score pass has no merge cost per split: about four waves of CTAs
+  int64_t ss = (4LL * sm_count() + pl->n_groups - 1) / pl->n_groups;
+  ss = std::max<int64_t>(1, std::min<int64_t>(ss, tiles));
+  int64_t sper = (L + ss - 1) / ss;
+  sper = (sper + kTile - 1) / kTile * kTile;
+  pl->score_splits = (int)((L + sper - 1) / sper);
+  pl->score_keys = (int)sper;
   size_t off = 0;
   pl->off_part_o = off;
   off = align_up(off + (size_t)pl->n_groups * splits * kRows * D * 4, 256);
@@ -125,17 +132,21 @@ hs2_status run_full(const CUtensorMap& km, const CUtensorMap& vm, const FullAttn
                     const FullPlan& pl, const SelectParams& sp, cudaStream_t s) {
   using SM = FullAttnSmem<D, FP8>;
   auto kp = attn_partial_kernel<D, FP8>;
-  auto ks = attn_score_kernel<D, FP8>;
+  auto ks = fp.G == 1 ? attn_score_kernel<D, FP8, 1>
+                      : (fp.G == 2 ? attn_score_kernel<D, FP8, 2> : attn_score_kernel<D, FP8, 4>);
   if (!set_smem(kp, SM::kBytes) || !set_smem(ks, SM::kScoreBytes)) return HS2_ERR_CUDA;
-  const int ctas = pl.n_groups * pl.n_splits;
-  kp<<<ctas, 160, SM::kBytes, s>>>(km, vm, fp);
+  kp<<<pl.n_groups * pl.n_splits, 160, SM::kBytes, s>>>(km, vm, fp);
   if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  const long long warps = (long long)pl.n_groups * kRows;
-  attn_combine_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(fp);
+  ks<<<pl.n_groups * pl.score_splits, 160, SM::kScoreBytes, s>>>(km, fp);
   if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  ks<<<ctas, 160, SM::kScoreBytes, s>>>(km, fp);
-  if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  select_topk_kernel<<<(unsigned)(fp.B * fp.T), kSelThreads, 0, s>>>(sp);
+  const long long nc_max = fp.L - fp.window + 1;  // candidates of the last query
+  if (nc_max <= kSelSmemMax) {
+    const int bytes = (int)std::max<long long>(16, nc_max * 4);
+    if (!set_smem(select_topk_kernel<true>, bytes)) return HS2_ERR_CUDA;
+    select_topk_kernel<true><<<(unsigned)(fp.B * fp.T), kSelThreads, bytes, s>>>(sp);
+  } else {
+    select_topk_kernel<false><<<(unsigned)(fp.B * fp.T), kSelThreads, 0, s>>>(sp);
+  }
   return launch_status();
 }
 
@@ -251,6 +262,8 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
   fp.groups_per_seq = pl.groups_per_seq;
   fp.n_splits = pl.n_splits;
   fp.split_keys = pl.split_keys;
+  fp.score_splits = pl.score_splits;
+  fp.score_keys = pl.score_keys;
   fp.window = window;
   fp.scale_log2 = scale * kLog2e;
 

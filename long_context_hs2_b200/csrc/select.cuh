@@ -81,10 +81,17 @@ __device__ __forceinline__ void find_kth_bin(const unsigned* hist, int nbins, in
   __syncthreads();
 }
 
+// SMEM = true: the candidate scores of the row are first copied to dynamic
+// shared memory (rows of at most kSelSmemMax candidates), and every later pass
+// reads them there.  SMEM = false: passes read the row in global memory.
+constexpr int kSelSmemMax = 48 * 1024;
+
+template <bool SMEM>
 __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectParams p) {
   __shared__ unsigned hist[2048];
   __shared__ int warp_tot[72];
   __shared__ int res[2];
+  extern __shared__ unsigned row_s[];
   const long long row = blockIdx.x;
   const int t = (int)(row % p.T);
   const long long i = p.L - p.T + t;
@@ -97,8 +104,20 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
     if (threadIdx.x == 0) p.n_sel[row] = (int32_t)n;
     return;
   }
-  const float* srow = p.score + row * p.L;
-  const unsigned* srow_u = reinterpret_cast<const unsigned*>(srow);
+  const unsigned* srow_u = reinterpret_cast<const unsigned*>(p.score + row * p.L);
+  if (SMEM) {
+    // 16-byte copies where the row start allows it (p.L % 4 == 0), else words
+    if ((p.L & 3) == 0) {
+      const uint4* g4 = reinterpret_cast<const uint4*>(srow_u);
+      uint4* s4 = reinterpret_cast<uint4*>(row_s);
+      for (long long j = threadIdx.x; j < nc / 4; j += kSelThreads) s4[j] = g4[j];
+      for (long long j = (nc / 4) * 4 + threadIdx.x; j < nc; j += kSelThreads) row_s[j] = srow_u[j];
+    } else {
+      for (long long j = threadIdx.x; j < nc; j += kSelThreads) row_s[j] = srow_u[j];
+    }
+    __syncthreads();
+    srow_u = row_s;
+  }
   int need = p.topk;
   unsigned prefix = 0;
   if (need > 0) {
@@ -130,32 +149,57 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
     need = res[1];
   }
   const unsigned tau = prefix;
-  // ordered compaction of {v > tau} and the first `need` of {v == tau}
-  int count = 0, eq_seen = 0;
+  // Ordered compaction of {v > tau} and the first `need` of {v == tau}.  Warp w
+  // owns the contiguous segment [w*seg, (w+1)*seg) of the candidates: a first
+  // pass counts its survivors (ballots), one block scan orders the warps, and a
+  // second pass writes each warp's survivors at its offset, in index order.
   if (p.topk > 0) {
-    for (long long base = 0; base < nc; base += kSelThreads) {
-      const long long j = base + threadIdx.x;
-      const unsigned v = j < nc ? srow_u[j] : 0u;
-      if (!__syncthreads_or(j < nc && v >= tau)) continue;  // nothing to keep here
-      const int gt = (j < nc && v > tau) ? 1 : 0;
-      const int eq = (j < nc && v == tau) ? 1 : 0;
-      int eq_rank;
-      const int eq_tot = block_exclusive_scan(eq, eq_rank, warp_tot);
-      const int sel = gt | ((eq && eq_seen + eq_rank < need) ? 1 : 0);
-      int pos;
-      const int sel_tot = block_exclusive_scan(sel, pos, warp_tot);
-      if (sel && count + pos < p.topk) out[count + pos] = (int32_t)j;
-      count += sel_tot;
-      eq_seen += eq_tot;
+    __shared__ int wsel[32], weq[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const long long seg = (nc + 31) / 32;
+    const long long s0 = warp * seg, s1 = min(nc, s0 + seg);
+    int n_gt = 0, n_eq = 0;
+    for (long long base = s0; base < s1; base += 32) {
+      const long long j = base + lane;
+      const unsigned v = j < s1 ? srow_u[j] : 0u;
+      n_gt += __popc(__ballot_sync(0xffffffffu, j < s1 && v > tau));
+      n_eq += __popc(__ballot_sync(0xffffffffu, j < s1 && v == tau));
     }
+    if (lane == 0) {
+      wsel[warp] = n_gt;
+      weq[warp] = n_eq;
+    }
+    __syncthreads();
+    int gt_before = 0, eq_before = 0;
+    for (int w = 0; w < warp; ++w) {
+      gt_before += wsel[w];
+      eq_before += weq[w];
+    }
+    // equal elements taken by this warp: those of rank < need overall
+    int pos = gt_before + min(eq_before, need);
+    int eq_rank = eq_before;
+    for (long long base = s0; base < s1; base += 32) {
+      const long long j = base + lane;
+      const unsigned v = j < s1 ? srow_u[j] : 0u;
+      const bool gt = j < s1 && v > tau;
+      const bool eq = j < s1 && v == tau;
+      const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+      const int my_eq_rank = eq_rank + __popc(eqm & ((1u << lane) - 1u));
+      const bool sel = gt || (eq && my_eq_rank < need);
+      const unsigned selm = __ballot_sync(0xffffffffu, sel);
+      if (sel) {
+        const int o = pos + __popc(selm & ((1u << lane) - 1u));
+        if (o < p.topk) out[o] = (int32_t)j;
+      }
+      pos += __popc(selm);
+      eq_rank += __popc(eqm);
+    }
+    if (warp == 31 && lane == 0 && pos != p.topk) raise_status(kStatusBadIndex);
   }
   const long long w0 = i - p.window + 1;
   for (int w = threadIdx.x; w < p.window; w += kSelThreads) out[p.topk + w] = (int32_t)(w0 + w);
   for (int s = p.topk + p.window + threadIdx.x; s < p.slots; s += kSelThreads) out[s] = -1;
-  if (threadIdx.x == 0) {
-    p.n_sel[row] = p.topk + p.window;
-    if (count != p.topk) raise_status(kStatusBadIndex);
-  }
+  if (threadIdx.x == 0) p.n_sel[row] = p.topk + p.window;
 }
 
 }  // namespace hs2

@@ -3,11 +3,13 @@
 //
 // One thread-block cluster of CS CTAs per query.  The query's selected slots
 // are cut into 64-slot tiles dealt round-robin to the cluster's CTAs; each CTA
-// gathers its tiles' K/V rows with 16-byte cp.async copies into 128B-swizzled
-// shared-memory tiles (a multi-stage ring), runs the warp attention core
-// (warps split every tile's keys 4 ways), merges its warps, and the cluster's
-// rank 0 merges the CTAs' partials through distributed shared memory.  No
-// global scratch is needed.
+// first copies (and range-checks) the positions of its slots into shared
+// memory, gathers its tiles' K/V rows with 16-byte cp.async copies into
+// 128B-swizzled shared-memory tiles (a multi-stage ring), runs the warp
+// attention core (warps split every tile's keys 4 ways) and merges its warps.
+// Then every CTA of the cluster merges one slice of the query's H x D output
+// from all CTAs' partials, read through distributed shared memory.  No global
+// scratch is needed.
 #pragma once
 
 #include "attn_warp.cuh"
@@ -46,8 +48,9 @@ struct SparseSmem {
   static constexpr int kMlOff = kQOff + kRowsQ * D * 2;
   static constexpr int kClOff = kMlOff + kSpWarps * kRowsQ * 8;  // CTA result: ml[rows], o[rows][D]
   static constexpr int kClBytes = kRowsQ * 8 + kRowsQ * D * 4;
-  static constexpr int kPosOff = kClOff + kClBytes;               // positions of the ring's tiles
-  static constexpr int kBytes = kPosOff + kStages * kSpTile * 4 + 1024;
+  static constexpr int kPosOff = kClOff + kClBytes;               // positions of the CTA's slots
+  static constexpr int kMaxSlots = 4096;
+  static constexpr int kBytes = kPosOff + kMaxSlots * 4 + 1024;
 };
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -64,48 +67,41 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+__device__ __forceinline__ float2 ld_dsmem_f32x2(uint32_t addr) {
+  float2 v;
+  asm("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
+  float4 v;
+  asm("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+      : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+      : "r"(addr));
   return v;
 }
 
-// Gathers the K/V rows of slots [slot0, slot0 + 64) into one ring stage and
-// records their positions (-1 = masked).  All 128 threads; one commit group.
+// Gathers the K/V rows of one 64-slot tile (positions pos[0..63], -1 =
+// masked) into a ring stage.  All 128 threads; one commit group.
 template <int D, bool FP8>
-__device__ __forceinline__ void sparse_gather_tile(const SparseParams& p, int b,
-                                                   const int32_t* sel, int n, int slot0,
-                                                   uint8_t* stage, int* pos_s) {
+__device__ __forceinline__ void sparse_gather_tile(const SparseParams& p, int b, const int* pos,
+                                                   uint8_t* stage) {
   constexpr int kRowBytes = D * (FP8 ? 1 : 2);
   constexpr int kChunks = kRowBytes / 16;
   constexpr int kTileBytes = kSpTile * kRowBytes;
-  for (int u = threadIdx.x; u < kSpTile; u += kSpWarps * 32) {
-    const int slot = slot0 + u;
-    int pos = -1;
-    if (slot < n) {
-      pos = sel[slot];
-      if (pos < 0 || (long long)pos >= p.L) {
-        raise_status(kStatusBadIndex);
-        pos = -1;
-      }
-    }
-    pos_s[u] = pos;
-  }
-  __syncthreads();
   const uint32_t dst0 = smem_u32(stage);
   for (int u = threadIdx.x; u < 2 * kSpTile * kChunks; u += kSpWarps * 32) {
     const int tsr = u / (kSpTile * kChunks);  // 0: K, 1: V
     const int rem = u % (kSpTile * kChunks);
     const int r = rem / kChunks, ch = rem % kChunks;
-    const int pos = pos_s[r];
+    const int ps = pos[r];
     const uint8_t* base = tsr ? p.v : p.k;
-    const uint8_t* src = base + ((long long)b * p.L + (pos < 0 ? 0 : pos)) * kRowBytes + ch * 16;
+    const uint8_t* src = base + ((long long)b * p.L + (ps < 0 ? 0 : ps)) * kRowBytes + ch * 16;
     uint32_t off;
     if (FP8)
       off = (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
     else
       off = sw128_offset(r, ch * 16, kSpTile);
-    cp_async16(dst0 + tsr * kTileBytes + off, src, pos < 0 ? 0 : 16);
+    cp_async16(dst0 + tsr * kTileBytes + off, src, ps < 0 ? 0 : 16);
   }
   cp_async_commit();
 }
@@ -119,7 +115,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   float2* ml_s = reinterpret_cast<float2*>(smem + SM::kMlOff);
   float2* cl_ml = reinterpret_cast<float2*>(smem + SM::kClOff);
   float* cl_o = reinterpret_cast<float*>(smem + SM::kClOff + SM::kRowsQ * 8);
-  int* pos_ring = reinterpret_cast<int*>(smem + SM::kPosOff);
+  int* pos_all = reinterpret_cast<int*>(smem + SM::kPosOff);  // [my_tiles][64]
 
   const int cs = p.cs;
   const uint32_t rank = cs > 1 ? cluster_ctarank() : 0u;
@@ -146,12 +142,26 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   const float* ksc = FP8 ? p.k_scale + (long long)b * p.L : nullptr;
   const float* vsc = FP8 ? p.v_scale + (long long)b * p.L : nullptr;
 
+  // positions of this CTA's slots: tile k of the CTA is slot tile rank + k*cs
+  for (int u = threadIdx.x; u < my_tiles * kSpTile; u += 128) {
+    const int slot = ((int)rank + (u / kSpTile) * cs) * kSpTile + (u % kSpTile);
+    int ps = -1;
+    if (slot < n) {
+      ps = sel[slot];
+      if (ps < 0 || (long long)ps >= p.L) {
+        raise_status(kStatusBadIndex);
+        ps = -1;
+      }
+    }
+    pos_all[u] = ps;
+  }
+  __syncthreads();
+
   // prologue: fill kStages-1 ring slots
 #pragma unroll
   for (int s = 0; s < SM::kStages - 1; ++s) {
     if (s < my_tiles)
-      sparse_gather_tile<D, FP8>(p, b, sel, n, ((int)rank + s * cs) * kSpTile,
-                                 smem + s * SM::kStageBytes, pos_ring + s * kSpTile);
+      sparse_gather_tile<D, FP8>(p, b, pos_all + s * kSpTile, smem + s * SM::kStageBytes);
     else
       cp_async_commit();
   }
@@ -167,7 +177,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
     __syncthreads();
     const int s = k % SM::kStages;
     uint8_t* stage = smem + s * SM::kStageBytes;
-    const int* pos = pos_ring + s * kSpTile;
+    const int* pos = pos_all + k * kSpTile;
     uint32_t kt, vt;
     int key0, rows;
     if (FP8) {
@@ -205,8 +215,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
     const int kn = k + SM::kStages - 1;
     const int sn = kn % SM::kStages;
     if (kn < my_tiles)
-      sparse_gather_tile<D, FP8>(p, b, sel, n, ((int)rank + kn * cs) * kSpTile,
-                                 smem + sn * SM::kStageBytes, pos_ring + sn * kSpTile);
+      sparse_gather_tile<D, FP8>(p, b, pos_all + kn * kSpTile, smem + sn * SM::kStageBytes);
     else
       cp_async_commit();
   }
@@ -255,29 +264,47 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
       }
     cl_ml[r] = make_float2(M, lt);
   }
-  if (cs > 1) cluster_sync_all();
-  else __syncthreads();
-
-  if (rank == 0) {
-    // merge the cluster's CTAs (rank 0 reads the others' results in place)
-    const uint32_t ml_addr = smem_u32(cl_ml), o_addr = smem_u32(cl_o);
+  if (cs == 1) {
+    __syncthreads();
     for (int u = threadIdx.x; u < p.H * D; u += 128) {
-      const int r = u / D;
-      float M = kNegInf;
-      for (int q = 0; q < cs; ++q) M = fmaxf(M, ld_dsmem_f32(mapa_shared(ml_addr + r * 8, q)));
-      float lt = 0.f, acc = 0.f;
-      if (M != kNegInf)
-        for (int q = 0; q < cs; ++q) {
-          const float m = ld_dsmem_f32(mapa_shared(ml_addr + r * 8, q));
-          const float l = ld_dsmem_f32(mapa_shared(ml_addr + r * 8 + 4, q));
-          const float fct = (m == kNegInf) ? 0.f : fast_exp2(m - M);
-          lt += l * fct;
-          acc += fct * ld_dsmem_f32(mapa_shared(o_addr + u * 4, q));
-        }
-      p.o[qrow * p.H * D + u] = lt > 0.f ? acc / lt : 0.f;
+      const float2 v = cl_ml[u / D];
+      p.o[qrow * p.H * D + u] = v.y > 0.f ? cl_o[u] / v.y : 0.f;
     }
+    return;
   }
-  if (cs > 1) cluster_sync_all();  // keep every CTA's shared memory alive until rank 0 is done
+  cluster_sync_all();
+  // CTA `rank` merges elements [rank*chunk, (rank+1)*chunk) of the H x D output
+  // (chunk is a multiple of 4: H*D is a multiple of 512 and cs <= 8)
+  const int chunk = p.H * D / cs;
+  const uint32_t ml_addr = smem_u32(cl_ml), o_addr = smem_u32(cl_o);
+  for (int u = (int)rank * chunk + 4 * threadIdx.x; u < ((int)rank + 1) * chunk; u += 4 * 128) {
+    const int r = u / D;
+    float2 mls[8];
+    float M = kNegInf;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < cs) {
+        mls[q] = ld_dsmem_f32x2(mapa_shared(ml_addr + r * 8, q));
+        M = fmaxf(M, mls[q].x);
+      }
+    float lt = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < cs) {
+        const float4 o = ld_dsmem_f32x4(mapa_shared(o_addr + u * 4, q));
+        const float f = (M == kNegInf || mls[q].x == kNegInf) ? 0.f : fast_exp2(mls[q].x - M);
+        lt += mls[q].y * f;
+        acc.x += f * o.x;
+        acc.y += f * o.y;
+        acc.z += f * o.z;
+        acc.w += f * o.w;
+      }
+    const float inv = lt > 0.f ? 1.f / lt : 0.f;
+    *reinterpret_cast<float4*>(p.o + qrow * p.H * D + u) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+  cluster_sync_all();  // keep every CTA's shared memory alive until all reads are done
 }
 
 }  // namespace hs2
