@@ -1,0 +1,602 @@
+// Full-attention layer on the 5th-generation tensor cores (tcgen05), for
+// head_dim 128 and a bf16 cache.
+//
+// MQA: every query row of a group -- N rows = N/H queries x H heads -- reads
+// the same K/V stream.  Each 128-key tile is processed transposed:
+//   S^T[128 keys][N rows] = K_tile[128 x 128] . Q^T        (M = 128 keys)
+//   O^T[128 d][N rows]   += V_tile^T[128 d x 128 keys] . P (M = 128 d)
+// with fp32 accumulators in tensor memory (TMEM).  In S^T, TMEM lane = key, so
+// the thread that owns a lane holds one key's logits for all N rows: the
+// head-sum of the selection score needs no cross-thread step, and the softmax
+// exponentials are element-wise.  The softmax normaliser uses a lazily
+// refreshed per-row reference max (raised, and O and the row sums rescaled,
+// only when some logit exceeds it by more than 2^8), so the common tile needs
+// no cross-thread max; each thread keeps its keys' partial row sums in a TMEM
+// column block.
+//
+// Warp roles (192 threads): warp 0 issues the TMA loads of the K/V tile ring;
+// warp 1 allocates TMEM and one of its threads issues every tcgen05.mma; warps
+// 2-5 are the softmax warps (one TMEM lane = one key each).
+//   attn_tc_partial : per (group, split): reference max m, sum l and
+//                     un-normalised O of the split.
+//   attn_tc_score   : merges the splits into lse and O, then recomputes S^T per
+//                     tile and writes score_j = sum over a query's heads of
+//                     exp(s - lse), with the level-1 selection histogram.
+#pragma once
+
+#include "full_attn.cuh"
+#include "tc_common.cuh"
+
+namespace hs2 {
+
+constexpr int kTcKeys = 128;          // keys per tile (M of the score MMA)
+constexpr int kTcTileBytes = kTcKeys * 128 * 2;   // one bf16 K or V tile: 32 KB
+constexpr float kRescaleAbove = 8.f;  // base-2 logits may exceed the reference by this
+constexpr int kTcThreads = 192;
+
+// Shared-memory plan.  Partial kernel: K/V tile ring, Q, P^T (double-buffered
+// for N = 32), per-row reference max / correction / partial maxima and sums.
+template <int N>
+struct TcSmem {
+  static constexpr int kStages = N == 32 ? 3 : 2;
+  static constexpr int kNP = N == 32 ? 2 : 1;            // P^T buffers
+  static constexpr int kStageBytes = 2 * kTcTileBytes;   // K then V
+  static constexpr int kQOff = kStages * kStageBytes;
+  static constexpr int kQBytes = N * 256;
+  static constexpr int kPOff = kQOff + kQBytes;          // P^T [N rows][128 keys] bf16
+  static constexpr int kPBytes = N * 256;
+  static constexpr int kMrefOff = kPOff + kNP * kPBytes; // float [N]
+  static constexpr int kCorrOff = kMrefOff + N * 4;      // float [N]
+  static constexpr int kTmaxOff = kCorrOff + N * 4;      // float [4][N] (also the row sums)
+  static constexpr int kBarOff = kTmaxOff + 4 * N * 4;
+  static constexpr int kNumBars = 2 * kStages + 4 + 2 * kNP;
+  static constexpr int kSlotOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kSlotOff + 16 + 1024;
+  // score kernel: K-only ring, staged (m, l) partials of the group, Q, histograms
+  static constexpr int kSStages = N == 32 ? 4 : 3;
+  static constexpr int kSMlOff = kSStages * kTcTileBytes;
+  static constexpr int kSMlBytes = 32 * 1024;            // rows x splits x 8 bytes
+  static constexpr int kSQOff = kSMlOff + kSMlBytes;
+  static constexpr int kSHistOff = kSQOff + kQBytes;
+  static constexpr int kSHistBytes = (N == 32 ? 4 : 4) * kHistBins * 4;
+  static constexpr int kSLseOff = kSHistOff + kSHistBytes;
+  static constexpr int kSBarOff = kSLseOff + N * 4;
+  static constexpr int kSSlotOff = kSBarOff + (2 * kSStages + 4) * 8;
+  static constexpr int kSBytes = kSSlotOff + 16 + 1024;
+};
+
+// Barrier, and block-wide OR, over the softmax warps (named barrier 1).
+template <int kThreads>
+__device__ __forceinline__ void softmax_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+}
+template <int kThreads>
+__device__ __forceinline__ bool softmax_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kThreads)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Loads the group's N query rows (row r = query t0 + r/H, head r%H) into a
+// K-major 128B-swizzled bf16 tile (two 64-column halves of N rows); rows of
+// queries past T are zero.  Called by all threads of the CTA.
+template <int N>
+__device__ __forceinline__ void tc_load_q(const FullAttnParams& p, int b, int t0, uint8_t* qs) {
+  for (int u = threadIdx.x; u < N * 16; u += blockDim.x) {
+    const int r = u >> 4, ch = u & 15;
+    const int t = t0 + r / p.H, h = r % p.H;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (t < p.T)
+      v = *reinterpret_cast<const uint4*>(p.q + (((long long)b * p.T + t) * p.H + h) * 128 + ch * 8);
+    *reinterpret_cast<uint4*>(qs + sw128_offset(r, ch * 16, N)) = v;
+  }
+}
+
+// Issues the 8 MMAs of S^T[128 x N] = K_tile . Q^T into TMEM column `d_col`.
+template <int N>
+__device__ __forceinline__ void tc_issue_qk(uint32_t tmem_d, uint32_t k_addr, uint32_t q_addr) {
+  constexpr uint32_t idesc = tc_idesc_f16(128, N, kTcBF16, false, false);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const uint32_t half = ks >> 2, koff = (ks & 3) * 32;
+    tc_mma_f16(tmem_d, sw128_kmajor_desc(k_addr + half * (kTcKeys * 128) + koff),
+               sw128_kmajor_desc(q_addr + half * (N * 128) + koff), idesc, ks > 0);
+  }
+}
+
+// Issues the 8 MMAs of O^T[128 x N] (+)= V_tile^T . P, V read MN-major from its
+// TMA tile (d contiguous within a 64-d half, halves 16 KB apart), P^T K-major.
+template <int N>
+__device__ __forceinline__ void tc_issue_pv(uint32_t tmem_d, uint32_t v_addr, uint32_t p_addr,
+                                            bool accumulate) {
+  constexpr uint32_t idesc = tc_idesc_f16(128, N, kTcBF16, true, false);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const uint32_t half = ks >> 2, koff = (ks & 3) * 32;
+    tc_mma_f16(tmem_d, sw128_mnmajor_desc(v_addr + ks * 16 * 128, kTcKeys * 128),
+               sw128_kmajor_desc(p_addr + half * (N * 128) + koff), idesc,
+               accumulate || ks > 0);
+  }
+}
+
+// Partial kernel: warps 0 (TMA), 1 (MMA) and 8 softmax warps 2-9.  Softmax
+// warp w reads TMEM lane quarter w%4 (keys, or d for O^T) and the column half
+// (w-2)/4 of the N rows, so two warps share each scheduler and each thread
+// handles one key x N/2 rows per tile.
+constexpr int kTcPartialThreads = 320;
+constexpr int kTcSoftmax = 256;
+
+template <int N, int G>
+__global__ void __launch_bounds__(kTcPartialThreads, 1)
+    attn_tc_partial_kernel(const __grid_constant__ CUtensorMap kmap,
+                           const __grid_constant__ CUtensorMap vmap, const FullAttnParams p) {
+  using SM = TcSmem<N>;
+  constexpr int S = SM::kStages;
+  constexpr int NP = SM::kNP;
+  constexpr int kH = N / G;     // heads per query
+  constexpr int NC = N / 2;     // columns per softmax warp
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  float* m_ref = reinterpret_cast<float*>(smem + SM::kMrefOff);
+  float* corr = reinterpret_cast<float*>(smem + SM::kCorrOff);
+  float* tmax = reinterpret_cast<float*>(smem + SM::kTmaxOff);
+  uint64_t* kv_full = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
+  uint64_t* kv_empty = kv_full + S;
+  uint64_t* s_full = kv_empty + S;   // [2]
+  uint64_t* s_empty = s_full + 2;    // [2]
+  uint64_t* p_full = s_empty + 2;    // [NP]
+  uint64_t* pv_done = p_full + NP;   // [NP]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kSlotOff);
+
+  const int split = blockIdx.x % p.n_splits;
+  const int grp = blockIdx.x / p.n_splits;
+  const int b = grp / p.groups_per_seq;
+  const int t0 = (grp % p.groups_per_seq) * G;
+  const int t_last = min(p.T, t0 + G) - 1;
+  const long long i_last = p.L - p.T + t_last;
+  const long long k_lo = (long long)split * p.split_keys;
+  const long long k_hi = min(k_lo + p.split_keys, i_last + 1);
+  const long long part = (long long)grp * p.n_splits + split;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (split == 0) {  // clear the group's level-1 selection histograms
+    for (int u = threadIdx.x; u < G * kHistBins; u += blockDim.x) {
+      const int t = t0 + u / kHistBins;
+      if (t < p.T) p.hist[((long long)b * p.T + t) * kHistBins + (u % kHistBins)] = 0u;
+    }
+  }
+  if (k_lo >= k_hi) {  // empty split: neutral partial
+    for (int u = threadIdx.x; u < N * 128; u += blockDim.x) p.part_o[part * N * 128 + u] = 0.f;
+    if (threadIdx.x < N) p.part_ml[part * N + threadIdx.x] = make_float2(kNegInf, 0.f);
+    return;
+  }
+  const int n_tiles = (int)((k_hi - k_lo + kTcKeys - 1) / kTcKeys);
+
+  tc_load_q<N>(p, b, t0, smem + SM::kQOff);
+  if (threadIdx.x < N) m_ref[threadIdx.x] = kNegInf;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], kTcSoftmax / 32);
+    }
+    for (int i = 0; i < NP; ++i) {
+      mbar_init(&p_full[i], kTcSoftmax / 32);
+      mbar_init(&pv_done[i], 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 4 * N);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();  // Q (generic-proxy writes) is read by the tensor cores
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t q_addr = smem_u32(smem + SM::kQOff);
+  const uint32_t p_addr = smem_u32(smem + SM::kPOff);
+
+  if (warp == 0) {
+    // -------------------------------------------------------------- TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      const uint64_t pol_k = policy_evict_last(), pol_v = policy_evict_first();
+      for (int n = 0; n < n_tiles; ++n) {
+        const int s = n % S;
+        if (n >= S && !mbar_wait(&kv_empty[s], ((n / S) - 1) & 1)) break;
+        uint8_t* st = smem + s * SM::kStageBytes;
+        mbar_arrive_expect_tx(&kv_full[s], SM::kStageBytes);
+        const int row = (int)((long long)b * p.L + k_lo + (long long)n * kTcKeys);
+        tma_load_2d(st, &kmap, &kv_full[s], 0, row, pol_k);
+        tma_load_2d(st + 16384, &kmap, &kv_full[s], 64, row, pol_k);
+        tma_load_2d(st + kTcTileBytes, &vmap, &kv_full[s], 0, row, pol_v);
+        tma_load_2d(st + kTcTileBytes + 16384, &vmap, &kv_full[s], 64, row, pol_v);
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- MMA
+    if (lane == 0) {
+      bool ok = true;
+      auto pv = [&](int m) {
+        if (!mbar_wait(&p_full[m % NP], (m / NP) & 1)) return false;
+        tc_fence_after();
+        tc_issue_pv<N>(tmem + 2 * N, smem_u32(smem + (m % S) * SM::kStageBytes + kTcTileBytes),
+                       p_addr + (m % NP) * SM::kPBytes, m > 0);
+        tc_commit(&pv_done[m % NP]);
+        tc_commit(&kv_empty[m % S]);
+        return true;
+      };
+      for (int n = 0; n < n_tiles && ok; ++n) {
+        const int s = n % S, bb = n & 1;
+        if (!mbar_wait(&kv_full[s], (n / S) & 1)) break;
+        if (n >= 2 && !mbar_wait(&s_empty[bb], ((n - 2) >> 1) & 1)) break;
+        tc_fence_after();
+        tc_issue_qk<N>(tmem + bb * N, smem_u32(smem + s * SM::kStageBytes), q_addr);
+        tc_commit(&s_full[bb]);
+        if (n >= 1) ok = pv(n - 1);
+      }
+      if (ok) pv(n_tiles - 1);
+    }
+  } else {
+    // ---------------------------------------------------------- softmax
+    const int wq = warp & 3;                 // TMEM lane quarter
+    const int c0 = ((warp - 2) >> 2) * NC;   // first of this warp's NC columns
+    const int st = threadIdx.x - 64;         // softmax thread 0..255
+    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+    const int keyrow = wq * 32 + lane;       // row of S^T (key) / of O^T (d)
+    const float sl = p.scale_log2;
+    // P^T store address of (row c0 + c, this key): base + c*128 + xoff[(c0 + c) & 7]
+    uint8_t* p_base = smem + SM::kPOff + (keyrow >> 6) * (N * 128) + c0 * 128;
+    uint32_t xoff[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) xoff[m] = ((((keyrow & 63) >> 3) ^ m) << 4) + (keyrow & 7) * 2;
+    bool failed = false;
+    {  // TMEM is undefined at allocation: clear this thread's row sums
+      float z[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) z[i] = 0.f;
+#pragma unroll
+      for (int c = 0; c < NC; c += 16) tmem_st16(tmem + lane_base + 3 * N + c0 + c, z);
+      tmem_st_wait();
+    }
+    for (int n = 0; n < n_tiles; ++n) {
+      const int bb = n & 1;
+      failed |= !mbar_wait(&s_full[bb], (n >> 1) & 1);
+      tc_fence_after();
+      const long long key0 = k_lo + (long long)n * kTcKeys;
+      const long long j = key0 + keyrow;
+      // a tile is "full" when every key is in range and causal for every query
+      const bool full_tile = key0 + kTcKeys <= k_hi && key0 + kTcKeys - 1 <= p.L - p.T + t0;
+      // limit[q]: last key query q of the group may see (in range of this split)
+      long long limit[G];
+#pragma unroll
+      for (int q = 0; q < G; ++q) limit[q] = min(k_hi - 1, p.L - p.T + t0 + q);
+      const uint32_t s_addr = tmem + lane_base + bb * N + c0;
+      // sweep 1: does any logit exceed its row's reference by more than 2^8?
+      bool need = false;
+#pragma unroll
+      for (int c = 0; c < NC; c += 16) {
+        float x[16];
+        tmem_ld16(s_addr + c, x);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int col = c0 + c + i;
+          const bool ok = full_tile || j <= limit[(c + i) / kH + c0 / kH];
+          need |= ok && x[i] * sl > m_ref[col] + kRescaleAbove;
+        }
+      }
+      if (n >= NP) {  // the P^T buffer of this tile is free once PV(n - NP) is done
+        failed |= !mbar_wait(&pv_done[n % NP], ((n - NP) / NP) & 1);
+        tc_fence_after();
+      }
+      const bool any_need = softmax_any<kTcSoftmax>(need);
+      if (softmax_any<kTcSoftmax>(failed)) break;
+      if (any_need) {
+        // new reference: column max of this tile's logits (and the old reference)
+#pragma unroll
+        for (int c = 0; c < NC; c += 16) {
+          float x[16];
+          tmem_ld16(s_addr + c, x);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const bool ok = full_tile || j <= limit[(c + i) / kH + c0 / kH];
+            const float v = warp_max(ok ? x[i] * sl : kNegInf);
+            if (lane == 0) tmax[wq * N + c0 + c + i] = v;
+          }
+        }
+        softmax_sync<kTcSoftmax>();
+        if (st < N) {
+          const float mo = m_ref[st];
+          const float mn = fmaxf(fmaxf(mo, fmaxf(tmax[st], tmax[N + st])),
+                                 fmaxf(tmax[2 * N + st], tmax[3 * N + st]));
+          corr[st] = (mn == kNegInf) ? 1.f : fast_exp2(mo - mn);
+          m_ref[st] = mn;
+        }
+        softmax_sync<kTcSoftmax>();
+        if (n >= 1) {  // O^T is rescaled once PV(n - 1) is done
+          failed |= !mbar_wait(&pv_done[(n - 1) % NP], ((n - 1) / NP) & 1);
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int c = 0; c < NC; c += 16) {
+          float v[16];
+          tmem_ld16(tmem + lane_base + 3 * N + c0 + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] *= corr[c0 + c + i];
+          tmem_st16(tmem + lane_base + 3 * N + c0 + c, v);
+          if (n >= 1) {
+            tmem_ld16(tmem + lane_base + 2 * N + c0 + c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] *= corr[c0 + c + i];
+            tmem_st16(tmem + lane_base + 2 * N + c0 + c, v);
+          }
+        }
+      }
+      // sweep 2: p = 2^(x - m_ref), row sums, P^T (bf16) for the PV product
+      uint8_t* pt = p_base + (n % NP) * SM::kPBytes;
+#pragma unroll
+      for (int c = 0; c < NC; c += 16) {
+        float x[16], lv[16];
+        tmem_ld16(s_addr + c, x);
+        tmem_ld16(tmem + lane_base + 3 * N + c0 + c, lv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int col = c0 + c + i;
+          const bool ok = full_tile || j <= limit[(c + i) / kH + c0 / kH];
+          const float mr = m_ref[col];
+          const float pr = (ok && mr != kNegInf) ? fast_exp2(x[i] * sl - mr) : 0.f;
+          lv[i] += pr;
+          *reinterpret_cast<__nv_bfloat16*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
+              __float2bfloat16_rn(pr);
+        }
+        tmem_st16(tmem + lane_base + 3 * N + c0 + c, lv);
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s_empty[bb]);
+        mbar_arrive(&p_full[n % NP]);
+      }
+    }
+    // ------------------------------------------------------- epilogue
+    failed |= !mbar_wait(&pv_done[(n_tiles - 1) % NP], ((n_tiles - 1) / NP) & 1);
+    tc_fence_after();
+    if (!softmax_any<kTcSoftmax>(failed)) {
+      float* lsum = tmax;  // [4 quarters][N]
+#pragma unroll
+      for (int c = 0; c < NC; c += 16) {
+        float v[16];
+        tmem_ld16(tmem + lane_base + 3 * N + c0 + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float s = warp_sum(v[i]);
+          if (lane == 0) lsum[wq * N + c0 + c + i] = s;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < NC; c += 16) {
+        float v[16];
+        tmem_ld16(tmem + lane_base + 2 * N + c0 + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p.part_o[(part * N + c0 + c + i) * 128 + keyrow] = v[i];
+      }
+      softmax_sync<kTcSoftmax>();
+      if (st < N) {
+        const float lt = lsum[st] + lsum[N + st] + lsum[2 * N + st] + lsum[3 * N + st];
+        p.part_ml[part * N + st] = make_float2(m_ref[st], lt);
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 4 * N);
+  }
+}
+
+template <int N, int G>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_tc_score_kernel(const __grid_constant__ CUtensorMap kmap, const FullAttnParams p) {
+  using SM = TcSmem<N>;
+  constexpr int S = SM::kSStages;
+  constexpr int kH = N / G;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  float2* ml_s = reinterpret_cast<float2*>(smem + SM::kSMlOff);  // [N][n_splits]
+  unsigned* hist_s = reinterpret_cast<unsigned*>(smem + SM::kSHistOff);
+  float* lse2_s = reinterpret_cast<float*>(smem + SM::kSLseOff);
+  uint64_t* kv_full = reinterpret_cast<uint64_t*>(smem + SM::kSBarOff);
+  uint64_t* kv_empty = kv_full + S;
+  uint64_t* s_full = kv_empty + S;  // [2]
+  uint64_t* s_empty = s_full + 2;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kSSlotOff);
+
+  const int split = blockIdx.x % p.score_splits;
+  const int grp = blockIdx.x / p.score_splits;
+  const int b = grp / p.groups_per_seq;
+  const int t0 = (grp % p.groups_per_seq) * G;
+  const int t_last = min(p.T, t0 + G) - 1;
+  const long long i_last = p.L - p.T + t_last;
+  const long long k_lo = (long long)split * p.score_keys;
+  const long long k_hi = min(k_lo + p.score_keys, i_last - p.window + 1);
+  const int n_tiles = k_lo < k_hi ? (int)((k_hi - k_lo + kTcKeys - 1) / kTcKeys) : 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ns = p.n_splits;
+
+  // stage the group's (m, l) partials; clear the histograms; load Q
+  {
+    const float2* ml_g = p.part_ml + (long long)grp * ns * N;
+    for (int u = threadIdx.x; u < N * ns; u += kTcThreads) {
+      const int sp = u / N, r = u % N;
+      ml_s[r * ns + sp] = ml_g[(long long)sp * N + r];
+    }
+  }
+  for (int u = threadIdx.x; u < G * kHistBins; u += kTcThreads) hist_s[u] = 0u;
+  if (n_tiles > 0) tc_load_q<N>(p, b, t0, smem + SM::kSQOff);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1 && n_tiles > 0) {
+    tmem_alloc(tmem_slot, 2 * N);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = n_tiles > 0 ? *tmem_slot : 0u;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&kmap);
+      const uint64_t pol = policy_evict_first();
+      for (int n = 0; n < n_tiles; ++n) {
+        const int s = n % S;
+        if (n >= S && !mbar_wait(&kv_empty[s], ((n / S) - 1) & 1)) break;
+        uint8_t* st = smem + s * kTcTileBytes;
+        mbar_arrive_expect_tx(&kv_full[s], kTcTileBytes);
+        const int row = (int)((long long)b * p.L + k_lo + (long long)n * kTcKeys);
+        tma_load_2d(st, &kmap, &kv_full[s], 0, row, pol);
+        tma_load_2d(st + 16384, &kmap, &kv_full[s], 64, row, pol);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(smem + SM::kSQOff);
+      for (int n = 0; n < n_tiles; ++n) {
+        const int s = n % S, bb = n & 1;
+        if (!mbar_wait(&kv_full[s], (n / S) & 1)) break;
+        if (n >= 2 && !mbar_wait(&s_empty[bb], ((n - 2) >> 1) & 1)) break;
+        tc_fence_after();
+        tc_issue_qk<N>(tmem + bb * N, smem_u32(smem + s * kTcTileBytes), q_addr);
+        tc_commit(&s_full[bb]);
+        tc_commit(&kv_empty[s]);
+      }
+    }
+  } else {
+    // ---- score warps: lse (base 2) of the group's rows, merged over the splits
+    const int st = threadIdx.x - 64;
+    for (int r = st; r < N; r += 128) {
+      float M = kNegInf;
+      for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, ml_s[r * ns + sp].x);
+      float lt = 0.f;
+      if (M != kNegInf)
+        for (int sp = 0; sp < ns; ++sp) {
+          const float2 v = ml_s[r * ns + sp];
+          lt += v.x == kNegInf ? 0.f : v.y * fast_exp2(v.x - M);
+        }
+      lse2_s[r] = M + log2f(lt);
+    }
+    softmax_sync<128>();
+    const int wq = warp & 3;
+    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+    const int keyrow = wq * 32 + lane;
+    const float sl = p.scale_log2;
+    for (int n = 0; n < n_tiles; ++n) {
+      const int bb = n & 1;
+      if (!mbar_wait(&s_full[bb], (n >> 1) & 1)) break;
+      tc_fence_after();
+      const long long j = k_lo + (long long)n * kTcKeys + keyrow;
+      float acc[G];
+#pragma unroll
+      for (int q = 0; q < G; ++q) acc[q] = 0.f;
+#pragma unroll
+      for (int c = 0; c < N / 32; ++c) {
+        float x[32];
+        tmem_ld32(tmem + lane_base + bb * N + 32 * c, x);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          acc[(32 * c + i) / kH] += fast_exp2(x[i] * sl - lse2_s[32 * c + i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[bb]);
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        const int t = t0 + q;
+        if (t < p.T && j <= p.L - p.T + t - p.window) {
+          p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
+          atomicAdd(&hist_s[q * kHistBins + (__float_as_uint(acc[q]) >> kHistShift)], 1u);
+        }
+      }
+    }
+    softmax_sync<128>();
+    for (int u = st; u < G * kHistBins; u += 128) {
+      const unsigned cnt = hist_s[u];
+      const int t = t0 + u / kHistBins;
+      if (cnt && t < p.T) atomicAdd(&p.hist[((long long)b * p.T + t) * kHistBins + (u % kHistBins)], cnt);
+    }
+    // ---- O and lse of row r, merged by the CTA whose score-split index is r mod score_splits
+    for (int r = warp - 2; r < N; r += 4) {
+      const int t = t0 + r / kH;
+      if (t >= p.T || (r % p.score_splits) != split) continue;
+      const float l2 = lse2_s[r];
+      const long long li = ((long long)b * p.T + t) * p.H + r % kH;
+      if (lane == 0) {
+        p.lse[li] = l2 * 0.69314718055994531f;
+        if (p.lse_out) p.lse_out[li] = l2 * 0.69314718055994531f;
+      }
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const float* po = p.part_o + ((long long)grp * ns * N + r) * 128;
+#pragma unroll 4
+      for (int sp = 0; sp < ns; ++sp) {
+        const float2 v = ml_s[r * ns + sp];
+        const float f = (v.x == kNegInf) ? 0.f : fast_exp2(v.x - l2);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[k] += f * po[(long long)sp * N * 128 + lane + 32 * k];
+      }
+      float* out = p.o + li * 128;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) out[lane + 32 * k] = acc[k];
+    }
+  }
+  __syncthreads();
+  if (warp == 1 && n_tiles > 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * N);
+  }
+}
+
+}  // namespace hs2

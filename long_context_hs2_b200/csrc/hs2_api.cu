@@ -9,6 +9,7 @@
 
 #include "bridge_gemm.cuh"
 #include "full_attn.cuh"
+#include "attn_tc.cuh"
 #include "select.cuh"
 #include "sparse_attn.cuh"
 
@@ -72,6 +73,9 @@ hs2_status launch_status() {
 
 // ------------------------------------------------ full-attention plan --
 struct FullPlan {
+  bool tc;       // tcgen05 path (D = 128, bf16 cache)
+  int rows;      // query rows per group (N of the tcgen05 tiles, or 32)
+  int tile;      // keys per pipeline tile
   int G, groups_per_seq, n_groups, n_splits, split_keys, score_splits, score_keys;
   size_t off_part_o, off_part_ml, off_lse, off_hist, off_score, total;
 };
@@ -84,33 +88,34 @@ bool check_attn_shape(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt) {
   return true;
 }
 
-bool make_full_plan(int B, int T, int64_t L, int H, int D, int topk, int window, FullPlan* pl) {
-  (void)topk;
-  (void)window;
-  pl->G = kRows / H;
+bool make_full_plan(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt, FullPlan* pl) {
+  pl->tc = D == 128 && dt == HS2_KV_BF16;
+  pl->rows = pl->tc && H == 32 && T >= 4 ? 128 : 32;
+  pl->tile = pl->tc ? kTcKeys : kTile;
+  pl->G = pl->rows / H;
   pl->groups_per_seq = (T + pl->G - 1) / pl->G;
   pl->n_groups = B * pl->groups_per_seq;
-  const int64_t tiles = (L + kTile - 1) / kTile;
-  const int64_t target = sm_count();  // about one wave of CTAs
-  int64_t splits = (target + pl->n_groups - 1) / pl->n_groups;
-  splits = std::max<int64_t>(1, std::min<int64_t>(splits, tiles));
-  int64_t per = (L + splits - 1) / splits;
-  per = (per + kTile - 1) / kTile * kTile;
-  splits = (L + per - 1) / per;
-  pl->n_splits = (int)splits;
-  pl->split_keys = (int)per;
-  // the score pass has no merge cost per split: about four waves of CTAs
-  int64_t ss = (4LL * sm_count() + pl->n_groups - 1) / pl->n_groups;
-  ss = std::max<int64_t>(1, std::min<int64_t>(ss, tiles));
-  int64_t sper = (L + ss - 1) / ss;
-  sper = (sper + kTile - 1) / kTile * kTile;
-  pl->score_splits = (int)((L + sper - 1) / sper);
-  pl->score_keys = (int)sper;
+  const int64_t tiles = (L + pl->tile - 1) / pl->tile;
+  auto split = [&](int64_t target, int64_t max_splits, int* n_out, int* keys_out) {
+    int64_t sp = (target + pl->n_groups - 1) / pl->n_groups;
+    sp = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(sp, tiles), max_splits));
+    int64_t per = (L + sp - 1) / sp;
+    per = (per + pl->tile - 1) / pl->tile * pl->tile;
+    *n_out = (int)((L + per - 1) / per);
+    *keys_out = (int)per;
+  };
+  // partials: about one wave of CTAs (each merged later); score pass: more
+  // (the tcgen05 score kernel stages the group's (m, l) partials in 32 KB of
+  //  shared memory: rows x splits x 8 bytes)
+  split(sm_count(), pl->tc ? (32 << 10) / (8 * pl->rows) : tiles, &pl->n_splits,
+        &pl->split_keys);
+  split((pl->tc ? 1LL : 4LL) * sm_count(), tiles, &pl->score_splits, &pl->score_keys);
+  const int R = pl->rows;
   size_t off = 0;
   pl->off_part_o = off;
-  off = align_up(off + (size_t)pl->n_groups * splits * kRows * D * 4, 256);
+  off = align_up(off + (size_t)pl->n_groups * pl->n_splits * R * D * 4, 256);
   pl->off_part_ml = off;
-  off = align_up(off + (size_t)pl->n_groups * splits * kRows * 8, 256);
+  off = align_up(off + (size_t)pl->n_groups * pl->n_splits * R * 8, 256);
   pl->off_lse = off;
   off = align_up(off + (size_t)B * T * H * 4, 256);
   pl->off_hist = off;
@@ -127,6 +132,18 @@ bool set_smem(K kernel, int bytes) {
          cudaSuccess;
 }
 
+hs2_status run_select(const FullAttnParams& fp, const SelectParams& sp, cudaStream_t s) {
+  const long long nc_max = fp.L - fp.window + 1;  // candidates of the last query
+  if (nc_max <= kSelSmemMax) {
+    const int bytes = (int)std::max<long long>(16, nc_max * 4);
+    if (!set_smem(select_topk_kernel<true>, bytes)) return HS2_ERR_CUDA;
+    select_topk_kernel<true><<<(unsigned)(fp.B * fp.T), kSelThreads, bytes, s>>>(sp);
+  } else {
+    select_topk_kernel<false><<<(unsigned)(fp.B * fp.T), kSelThreads, 0, s>>>(sp);
+  }
+  return launch_status();
+}
+
 template <int D, bool FP8>
 hs2_status run_full(const CUtensorMap& km, const CUtensorMap& vm, const FullAttnParams& fp,
                     const FullPlan& pl, const SelectParams& sp, cudaStream_t s) {
@@ -139,14 +156,25 @@ hs2_status run_full(const CUtensorMap& km, const CUtensorMap& vm, const FullAttn
   if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
   ks<<<pl.n_groups * pl.score_splits, 160, SM::kScoreBytes, s>>>(km, fp);
   if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  const long long nc_max = fp.L - fp.window + 1;  // candidates of the last query
-  if (nc_max <= kSelSmemMax) {
-    const int bytes = (int)std::max<long long>(16, nc_max * 4);
-    if (!set_smem(select_topk_kernel<true>, bytes)) return HS2_ERR_CUDA;
-    select_topk_kernel<true><<<(unsigned)(fp.B * fp.T), kSelThreads, bytes, s>>>(sp);
-  } else {
-    select_topk_kernel<false><<<(unsigned)(fp.B * fp.T), kSelThreads, 0, s>>>(sp);
-  }
+  return run_select(fp, sp, s);
+}
+
+template <int N>
+hs2_status run_full_tc(const CUtensorMap& km, const CUtensorMap& vm, const FullAttnParams& fp,
+                       const FullPlan& pl, cudaStream_t s) {
+  using SM = TcSmem<N>;
+  auto kp = N == 128 ? attn_tc_partial_kernel<N, 4>
+                     : (fp.G == 1 ? attn_tc_partial_kernel<N, 1>
+                                  : (fp.G == 2 ? attn_tc_partial_kernel<N, 2>
+                                               : attn_tc_partial_kernel<N, 4>));
+  auto ks = N == 128 ? attn_tc_score_kernel<N, 4>
+                     : (fp.G == 1 ? attn_tc_score_kernel<N, 1>
+                                  : (fp.G == 2 ? attn_tc_score_kernel<N, 2>
+                                               : attn_tc_score_kernel<N, 4>));
+  if (!set_smem(kp, SM::kBytes) || !set_smem(ks, SM::kSBytes)) return HS2_ERR_CUDA;
+  kp<<<pl.n_groups * pl.n_splits, kTcPartialThreads, SM::kBytes, s>>>(km, vm, fp);
+  if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+  ks<<<pl.n_groups * pl.score_splits, kTcThreads, SM::kSBytes, s>>>(km, fp);
   return launch_status();
 }
 
@@ -209,7 +237,7 @@ size_t hs2_full_attn_select_workspace(int B, int T, int64_t L, int H, int D, int
   if (!check_attn_shape(B, T, L, H, D, dt) || topk < 0 || window < 1 || topk + window > 4096)
     return 0;
   FullPlan pl;
-  make_full_plan(B, T, L, H, D, topk, window, &pl);
+  make_full_plan(B, T, L, H, D, dt, &pl);
   return pl.total;
 }
 
@@ -230,15 +258,15 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
   if (!check_attn_shape(B, T, L, H, D, dt) || topk + window > 4096) return HS2_ERR_UNSUPPORTED;
   if (dt == HS2_KV_FP8_E4M3 && D != 128) return HS2_ERR_UNSUPPORTED;
   FullPlan pl;
-  make_full_plan(B, T, L, H, D, topk, window, &pl);
+  make_full_plan(B, T, L, H, D, dt, &pl);
   if (!workspace || workspace_bytes < pl.total || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
 
   const bool fp8 = dt == HS2_KV_FP8_E4M3;
   const int elem = fp8 ? 1 : 2;
   CUtensorMap km, vm;
   const uint32_t box_cols = fp8 ? 128u : 64u;
-  if (!make_map_2d(&km, kv->k, (uint64_t)B * L, D, elem, box_cols, kTile) ||
-      !make_map_2d(&vm, kv->v, (uint64_t)B * L, D, elem, box_cols, kTile))
+  if (!make_map_2d(&km, kv->k, (uint64_t)B * L, D, elem, box_cols, pl.tile) ||
+      !make_map_2d(&vm, kv->v, (uint64_t)B * L, D, elem, box_cols, pl.tile))
     return HS2_ERR_CUDA;
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -279,6 +307,12 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
   sp.slots = topk + window;
 
   cudaStream_t s = (cudaStream_t)stream;
+  if (pl.tc) {
+    const hs2_status st =
+        pl.rows == 128 ? run_full_tc<128>(km, vm, fp, pl, s) : run_full_tc<32>(km, vm, fp, pl, s);
+    if (st != HS2_OK) return st;
+    return run_select(fp, sp, s);
+  }
   if (fp8) return run_full<128, true>(km, vm, fp, pl, sp, s);
   if (D == 128) return run_full<128, false>(km, vm, fp, pl, sp, s);
   return run_full<64, false>(km, vm, fp, pl, sp, s);

@@ -136,3 +136,10 @@ def test_sparse_out_of_range_index_is_reported():
                         tl.dev(nsel), 16, di.dt, O)
     assert hs2.hs2_last_device_status() == 6
     assert hs2.hs2_last_device_status() == 0   # cleared by the read
+
+
+def test_chunk_bf16_h32_wide_groups():
+    # several queries per sequence with 32 heads: groups of 4 queries x 32 heads
+    wl = WORKLOADS["decode_bf16_32k"].resized(B=2, T=70, L=9000, n_needles=20, n_sparse=1)
+    rows = np.unique(np.r_[0, 69, 70, 139, np.random.default_rng(2).integers(0, 140, 24)])
+    _check_block(wl, rows=rows)
