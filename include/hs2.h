@@ -163,6 +163,40 @@ HS2_API hs2_status hs2_sparse_attn(const void* Q, const hs2_kv_cache* kv, int B,
                            int slots, hs2_kv_dtype dt, float* O, hs2_stream_t stream);
 
 /*
+ * hs2_full_attn_select_noalloc -- hs2_full_attn_select for callers that
+ * cannot allocate device memory.  (The HySparse2 pages have no counterpart:
+ * this is a packaging choice of this library.)
+ *
+ * Some callers have no way to obtain a workspace: code hosted by a framework
+ * that reserves all device memory up front and hands its plugins no
+ * allocator, or code on a latency-critical path that cannot afford
+ * cudaMalloc's implicit device-wide synchronisation.  This entry point takes
+ * the same arguments as hs2_full_attn_select minus the workspace, and uses a
+ * scratch area built into the library instead: a static device array of
+ * HS2_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU which loads libhs2 keeps
+ * until the process exits.  It never calls cudaMalloc, cudaFree or any
+ * allocating routine.
+ *   - The first call on a device looks up that device's address of the array
+ *     (cudaGetSymbolAddress, with the caller's current device); make that
+ *     first call before any stream capture on the device.
+ *   - A request whose workspace (hs2_full_attn_select_workspace) exceeds
+ *     HS2_NOALLOC_SCRATCH_BYTES returns HS2_ERR_WORKSPACE and enqueues nothing.
+ *     For example, 8 sequences of 32K positions need about 3.6 MB.
+ *   - All calls on a device share the one array, and it keeps whatever the
+ *     last call left there; the kernels clear the parts that must start at
+ *     zero themselves.  Calls whose work overlaps on the GPU (different
+ *     streams, or different host threads) race on the array and must be
+ *     serialised by the caller.
+ * Outputs and status codes are those of hs2_full_attn_select.
+ */
+#define HS2_NOALLOC_SCRATCH_BYTES (16u << 20)
+HS2_API hs2_status hs2_full_attn_select_noalloc(const void* Q, const hs2_kv_cache* kv, int B,
+                                                int T, int64_t L, int H, int D, float scale,
+                                                int topk, int window, hs2_kv_dtype dt, float* O,
+                                                float* lse, int32_t* idx, int32_t* n_sel,
+                                                hs2_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the calling device's status
  * word: HS2_OK, HS2_ERR_TIMEOUT (a barrier wait gave up) or HS2_ERR_DEVICE
  * (an index was out of range).  HS2_ERR_CUDA if the wait itself failed.

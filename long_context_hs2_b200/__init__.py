@@ -24,7 +24,11 @@ _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error",
            4: "workspace", 5: "timeout", 6: "device index error"}
 
 EXPORTED = ("hs2_bridge_kv", "hs2_full_attn_select_workspace", "hs2_full_attn_select",
-            "hs2_sparse_attn", "hs2_last_device_status", "hs2_status_string", "hs2_version")
+            "hs2_full_attn_select_noalloc", "hs2_sparse_attn", "hs2_last_device_status",
+            "hs2_status_string", "hs2_version")
+
+# Size of the scratch area built into the library for hs2_full_attn_select_noalloc.
+HS2_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class Hs2Error(RuntimeError):
@@ -64,6 +68,9 @@ def load_library(path: str = LIB_PATH):
     lib.hs2_full_attn_select.restype = i32
     lib.hs2_full_attn_select.argtypes = [P, KV, i32, i32, i64, i32, i32, ctypes.c_float, i32, i32,
                                          i32, P, P, P, P, P, sz, P]
+    lib.hs2_full_attn_select_noalloc.restype = i32
+    lib.hs2_full_attn_select_noalloc.argtypes = [P, KV, i32, i32, i64, i32, i32, ctypes.c_float,
+                                                 i32, i32, i32, P, P, P, P, P]
     lib.hs2_sparse_attn.restype = i32
     lib.hs2_sparse_attn.argtypes = [P, KV, i32, i32, i64, i32, i32, ctypes.c_float, P, P, i32, i32,
                                     P, P]
@@ -130,6 +137,16 @@ def hs2_full_attn_select(Q, kv: hs2_kv_cache, B, T, L, H, D, scale, topk, window
         _ptr(Q), ctypes.byref(kv), int(B), int(T), int(L), int(H), int(D), float(scale), int(topk),
         int(window), int(dt), _ptr(O), _ptr(lse), _ptr(idx), _ptr(n_sel), _ptr(workspace),
         int(workspace_bytes), _stream(stream)))
+
+
+def hs2_full_attn_select_noalloc(Q, kv: hs2_kv_cache, B, T, L, H, D, scale, topk, window, dt,
+                                 O, lse, idx, n_sel, stream=None):
+    """hs2_full_attn_select without a workspace argument, for callers that cannot
+    allocate device memory; the library's built-in scratch area is used instead."""
+    _check("hs2_full_attn_select_noalloc", load_library().hs2_full_attn_select_noalloc(
+        _ptr(Q), ctypes.byref(kv), int(B), int(T), int(L), int(H), int(D), float(scale),
+        int(topk), int(window), int(dt), _ptr(O), _ptr(lse), _ptr(idx), _ptr(n_sel),
+        _stream(stream)))
 
 
 def hs2_sparse_attn(Q, kv: hs2_kv_cache, B, T, L, H, D, scale, idx, n_sel, slots, dt, O,

@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "bridge_gemm.cuh"
 #include "full_attn.cuh"
@@ -401,4 +402,54 @@ extern "C" hs2_status hs2_bridge_kv(const void* X, int64_t T, int hidden, const 
   const int grid = (int)std::min<long long>(tiles, sm_count());
   bridge_gemm_kernel<<<grid, kBrThreads, kBrSmemBytes, (cudaStream_t)stream>>>(xm, wm, p);
   return launch_status();
+}
+
+// ------------------------------------------------------------------------
+// Allocation-free variant of hs2_full_attn_select: the workspace is a static
+// device array compiled into the library (one per device, alive until the
+// process exits), shared by every call.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[HS2_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+
+// Device address of the scratch array on the current device, looked up once
+// per device (the host-side name of the array is only a stand-in: a kernel
+// handed it would fault or read the wrong memory).
+hs2_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HS2_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return HS2_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return HS2_ERR_CUDA;
+    }
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return HS2_OK;
+}
+
+}  // namespace
+
+extern "C" hs2_status hs2_full_attn_select_noalloc(const void* Q, const hs2_kv_cache* kv, int B,
+                                                   int T, int64_t L, int H, int D, float scale,
+                                                   int topk, int window, hs2_kv_dtype dt,
+                                                   float* O, float* lse, int32_t* idx,
+                                                   int32_t* n_sel, hs2_stream_t stream) {
+  const size_t need = hs2_full_attn_select_workspace(B, T, L, H, D, topk, window, dt);
+  if (need > HS2_NOALLOC_SCRATCH_BYTES) return HS2_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (need > 0) {  // need == 0: invalid shape, reported by the call below
+    const hs2_status st = noalloc_scratch(&scratch);
+    if (st != HS2_OK) return st;
+  }
+  return hs2_full_attn_select(Q, kv, B, T, L, H, D, scale, topk, window, dt, O, lse, idx, n_sel,
+                              scratch, need > 0 ? (size_t)HS2_NOALLOC_SCRATCH_BYTES : 0, stream);
 }
