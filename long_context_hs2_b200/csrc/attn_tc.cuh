@@ -49,7 +49,7 @@ struct TcSmem {
   static constexpr int kCorrOff = kMrefOff + N * 4;      // float [N]
   static constexpr int kTmaxOff = kCorrOff + N * 4;      // float [4][N] (also the row sums)
   static constexpr int kBarOff = kTmaxOff + 4 * N * 4;
-  static constexpr int kNumBars = 2 * kStages + 4 + 2 * kNP;
+  static constexpr int kNumBars = 2 * kStages + 5 + 2 * kNP;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kSlotOff + 16 + 1024;
   // score kernel: K-only ring, staged (m, l) partials of the group, Q, histograms
@@ -61,7 +61,7 @@ struct TcSmem {
   static constexpr int kSHistBytes = (N == 32 ? 4 : 4) * kHistBins * 4;
   static constexpr int kSLseOff = kSHistOff + kSHistBytes;
   static constexpr int kSBarOff = kSLseOff + N * 4;
-  static constexpr int kSSlotOff = kSBarOff + (2 * kSStages + 4) * 8;
+  static constexpr int kSSlotOff = kSBarOff + (2 * kSStages + 5) * 8;
   static constexpr int kSBytes = kSSlotOff + 16 + 1024;
 };
 
@@ -92,21 +92,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
-}
-
-// Loads the group's N query rows (row r = query t0 + r/H, head r%H) into a
-// K-major 128B-swizzled bf16 tile (two 64-column halves of N rows); rows of
-// queries past T are zero.  Called by all threads of the CTA.
-template <int N>
-__device__ __forceinline__ void tc_load_q(const FullAttnParams& p, int b, int t0, uint8_t* qs) {
-  for (int u = threadIdx.x; u < N * 16; u += blockDim.x) {
-    const int r = u >> 4, ch = u & 15;
-    const int t = t0 + r / p.H, h = r % p.H;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (t < p.T)
-      v = *reinterpret_cast<const uint4*>(p.q + (((long long)b * p.T + t) * p.H + h) * 128 + ch * 8);
-    *reinterpret_cast<uint4*>(qs + sw128_offset(r, ch * 16, N)) = v;
-  }
 }
 
 // Issues the 8 MMAs of S^T[128 x N] = K_tile . Q^T into TMEM column `d_col`.
@@ -163,6 +148,7 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
   uint64_t* s_empty = s_full + 2;    // [2]
   uint64_t* p_full = s_empty + 2;    // [NP]
   uint64_t* pv_done = p_full + NP;   // [NP]
+  uint64_t* q_ready = pv_done + NP;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kSlotOff);
 
   const int split = blockIdx.x % p.n_splits;
@@ -176,20 +162,18 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
   const long long part = (long long)grp * p.n_splits + split;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if (split == 0) {  // clear the group's level-1 selection histograms
-    for (int u = threadIdx.x; u < G * kHistBins; u += blockDim.x) {
-      const int t = t0 + u / kHistBins;
-      if (t < p.T) p.hist[((long long)b * p.T + t) * kHistBins + (u % kHistBins)] = 0u;
-    }
-  }
   if (k_lo >= k_hi) {  // empty split: neutral partial
+    if (split == 0)
+      for (int u = threadIdx.x; u < G * kHistBins; u += blockDim.x) {
+        const int t = t0 + u / kHistBins;
+        if (t < p.T) p.hist[((long long)b * p.T + t) * kHistBins + (u % kHistBins)] = 0u;
+      }
     for (int u = threadIdx.x; u < N * 128; u += blockDim.x) p.part_o[part * N * 128 + u] = 0.f;
     if (threadIdx.x < N) p.part_ml[part * N + threadIdx.x] = make_float2(kNegInf, 0.f);
     return;
   }
   const int n_tiles = (int)((k_hi - k_lo + kTcKeys - 1) / kTcKeys);
 
-  tc_load_q<N>(p, b, t0, smem + SM::kQOff);
   if (threadIdx.x < N) m_ref[threadIdx.x] = kNegInf;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -204,13 +188,13 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
       mbar_init(&p_full[i], kTcSoftmax / 32);
       mbar_init(&pv_done[i], 1);
     }
+    mbar_init(q_ready, kTcSoftmax / 32);
     fence_mbar_init();
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 4 * N);
     tmem_relinquish();
   }
-  fence_proxy_async_smem();  // Q (generic-proxy writes) is read by the tensor cores
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -249,6 +233,7 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
         tc_commit(&kv_empty[m % S]);
         return true;
       };
+      ok = mbar_wait(q_ready, 0);  // Q staged by the softmax warps
       for (int n = 0; n < n_tiles && ok; ++n) {
         const int s = n % S, bb = n & 1;
         if (!mbar_wait(&kv_full[s], (n / S) & 1)) break;
@@ -262,6 +247,23 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- softmax
+    // stage Q (read by the tensor cores: fence to the async proxy, then publish)
+    for (int u = threadIdx.x - 64; u < N * 16; u += kTcSoftmax) {
+      const int r = u >> 4, ch = u & 15;
+      const int t = t0 + r / p.H, h = r % p.H;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (t < p.T)
+        v = *reinterpret_cast<const uint4*>(p.q + (((long long)b * p.T + t) * p.H + h) * 128 + ch * 8);
+      *reinterpret_cast<uint4*>(smem + SM::kQOff + sw128_offset(r, ch * 16, N)) = v;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(q_ready);
+    if (split == 0)  // clear the group's level-1 selection histograms
+      for (int u = threadIdx.x - 64; u < G * kHistBins; u += kTcSoftmax) {
+        const int t = t0 + u / kHistBins;
+        if (t < p.T) p.hist[((long long)b * p.T + t) * kHistBins + (u % kHistBins)] = 0u;
+      }
     const int wq = warp & 3;                 // TMEM lane quarter
     const int c0 = ((warp - 2) >> 2) * NC;   // first of this warp's NC columns
     const int st = threadIdx.x - 64;         // softmax thread 0..255
@@ -442,6 +444,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* kv_empty = kv_full + S;
   uint64_t* s_full = kv_empty + S;  // [2]
   uint64_t* s_empty = s_full + 2;   // [2]
+  uint64_t* q_ready = s_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kSSlotOff);
 
   const int split = blockIdx.x % p.score_splits;
@@ -456,16 +459,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ns = p.n_splits;
 
-  // stage the group's (m, l) partials; clear the histograms; load Q
-  {
-    const float2* ml_g = p.part_ml + (long long)grp * ns * N;
-    for (int u = threadIdx.x; u < N * ns; u += kTcThreads) {
-      const int sp = u / N, r = u % N;
-      ml_s[r * ns + sp] = ml_g[(long long)sp * N + r];
-    }
-  }
-  for (int u = threadIdx.x; u < G * kHistBins; u += kTcThreads) hist_s[u] = 0u;
-  if (n_tiles > 0) tc_load_q<N>(p, b, t0, smem + SM::kSQOff);
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -475,13 +468,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 4);
     }
+    mbar_init(q_ready, 4);
     fence_mbar_init();
   }
   if (warp == 1 && n_tiles > 0) {
     tmem_alloc(tmem_slot, 2 * N);
     tmem_relinquish();
   }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -502,7 +495,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && n_tiles > 0 && mbar_wait(q_ready, 0)) {  // Q staged by the score warps
       const uint32_t q_addr = smem_u32(smem + SM::kSQOff);
       for (int n = 0; n < n_tiles; ++n) {
         const int s = n % S, bb = n & 1;
@@ -515,8 +508,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   } else {
-    // ---- score warps: lse (base 2) of the group's rows, merged over the splits
+    // ---- score warps: stage Q (for the tensor cores), the group's (m, l)
+    //      partials, clear the histograms; then lse (base 2) of the group's rows
     const int st = threadIdx.x - 64;
+    if (n_tiles > 0) {
+      for (int u = st; u < N * 16; u += 128) {
+        const int r = u >> 4, ch = u & 15;
+        const int t = t0 + r / p.H, h = r % p.H;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (t < p.T)
+          v = *reinterpret_cast<const uint4*>(p.q + (((long long)b * p.T + t) * p.H + h) * 128 + ch * 8);
+        *reinterpret_cast<uint4*>(smem + SM::kSQOff + sw128_offset(r, ch * 16, N)) = v;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
+    {
+      const float2* ml_g = p.part_ml + (long long)grp * ns * N;
+      for (int u = st; u < N * ns; u += 128) {
+        const int sp = u / N, r = u % N;
+        ml_s[r * ns + sp] = ml_g[(long long)sp * N + r];
+      }
+    }
+    for (int u = st; u < G * kHistBins; u += 128) hist_s[u] = 0u;
+    softmax_sync<128>();
     for (int r = st; r < N; r += 128) {
       float M = kNegInf;
       for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, ml_s[r * ns + sp].x);
@@ -568,28 +584,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int t = t0 + u / kHistBins;
       if (cnt && t < p.T) atomicAdd(&p.hist[((long long)b * p.T + t) * kHistBins + (u % kHistBins)], cnt);
     }
-    // ---- O and lse of row r, merged by the CTA whose score-split index is r mod score_splits
-    for (int r = warp - 2; r < N; r += 4) {
+    // ---- O and lse of row r, merged by the CTA whose score-split index is r mod
+    //      score_splits: thread st owns element d = st of the row
+    for (int r = split; r < N; r += p.score_splits) {
       const int t = t0 + r / kH;
-      if (t >= p.T || (r % p.score_splits) != split) continue;
+      if (t >= p.T) continue;
       const float l2 = lse2_s[r];
       const long long li = ((long long)b * p.T + t) * p.H + r % kH;
-      if (lane == 0) {
+      if (st == 0) {
         p.lse[li] = l2 * 0.69314718055994531f;
         if (p.lse_out) p.lse_out[li] = l2 * 0.69314718055994531f;
       }
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const float* po = p.part_o + ((long long)grp * ns * N + r) * 128;
-#pragma unroll 4
+      const float* po = p.part_o + ((long long)grp * ns * N + r) * 128 + st;
+      float acc = 0.f;
+#pragma unroll 8
       for (int sp = 0; sp < ns; ++sp) {
         const float2 v = ml_s[r * ns + sp];
         const float f = (v.x == kNegInf) ? 0.f : fast_exp2(v.x - l2);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[k] += f * po[(long long)sp * N * 128 + lane + 32 * k];
+        acc += f * po[(long long)sp * N * 128];
       }
-      float* out = p.o + li * 128;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) out[lane + 32 * k] = acc[k];
+      p.o[li * 128 + st] = acc;
     }
   }
   __syncthreads();

@@ -38,10 +38,11 @@ struct WarpAttn {
 
 // S[mt][nt] (raw dot products) of the warp's rows against 16 keys starting at
 // row `key0` of the key tile.  q_base/k_base are shared-memory addresses of
-// the Q tile (MT*16 rows) and of the key tile (rows_k rows per column half).
+// the Q tile (rows_q rows per column half; the warp's rows start at q_row0)
+// and of the key tile (rows_k rows per column half).
 template <int MT, int D>
 __device__ __forceinline__ void warp_qk(uint32_t q_base, uint32_t k_base, int key0, int rows_k,
-                                        float s[MT][2][4]) {
+                                        float s[MT][2][4], int q_row0 = 0, int rows_q = MT * 16) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
@@ -58,8 +59,8 @@ __device__ __forceinline__ void warp_qk(uint32_t q_base, uint32_t k_base, int ke
     uint32_t a[MT][4];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
-      ldsm_x4(q_base + sw128_offset(mt * 16 + qrow, ks * 32 + qcol, MT * 16), a[mt][0], a[mt][1],
-              a[mt][2], a[mt][3]);
+      ldsm_x4(q_base + sw128_offset(q_row0 + mt * 16 + qrow, ks * 32 + qcol, rows_q), a[mt][0],
+              a[mt][1], a[mt][2], a[mt][3]);
     uint32_t b0, b1, b2, b3;
     ldsm_x4(k_base + sw128_offset(krow, ks * 32 + kcol, rows_k), b0, b1, b2, b3);
 #pragma unroll
@@ -71,13 +72,14 @@ __device__ __forceinline__ void warp_qk(uint32_t q_base, uint32_t k_base, int ke
 }
 
 // Online-softmax update with base-2 logits x[mt][nt][e] (-inf = masked) and
-// O += P V for the 16 keys at row key0 of the value tile.  pv_scale[nt][j] is
-// the factor applied to p of key (nt*8 + 2c + j) before the PV product (the
+// O += P V for the 16 keys at row key0 of the value tile, over the D value
+// columns that start at byte column col0 of the tile.  pv_scale[nt][j] is the
+// factor applied to p of key (nt*8 + 2c + j) before the PV product (the
 // per-token E4M3 value scale; 1 for bf16).  l accumulates the unscaled p.
 template <int MT, int D>
 __device__ __forceinline__ void warp_softmax_pv(WarpAttn<MT, D>& st, float x[MT][2][4],
                                                 uint32_t v_base, int key0, int rows_v,
-                                                const float pv_scale[2][2]) {
+                                                const float pv_scale[2][2], int col0 = 0) {
   const int lane = threadIdx.x & 31;
   uint32_t pa[MT][4];
 #pragma unroll
@@ -118,7 +120,7 @@ __device__ __forceinline__ void warp_softmax_pv(WarpAttn<MT, D>& st, float x[MT]
 #pragma unroll
   for (int dp = 0; dp < D / 16; ++dp) {
     uint32_t b0, b1, b2, b3;
-    ldsm_x4_t(v_base + sw128_offset(vrow, dp * 32 + vcol, rows_v), b0, b1, b2, b3);
+    ldsm_x4_t(v_base + sw128_offset(vrow, col0 + dp * 32 + vcol, rows_v), b0, b1, b2, b3);
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
       mma_bf16_16816(st.o[mt][2 * dp], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b0, b1);
@@ -129,9 +131,11 @@ __device__ __forceinline__ void warp_softmax_pv(WarpAttn<MT, D>& st, float x[MT]
 
 // Converts `nkeys` rows (starting at row key0) of an E4M3 tile (128-byte
 // swizzled rows of D = 128 codes) into the bf16 swizzled layout of a tile
-// with rows_out rows per column half, rows renumbered from 0.  Whole warp.
+// with rows_out rows per column half, as its rows dst_row0 .. dst_row0+nkeys-1.
+// Whole warp.
 __device__ __forceinline__ void warp_fp8_rows_to_bf16(const uint8_t* src, int key0, int nkeys,
-                                                      uint8_t* dst, int rows_out) {
+                                                      uint8_t* dst, int rows_out,
+                                                      int dst_row0 = 0) {
   const int lane = threadIdx.x & 31;
   for (int u = lane; u < nkeys * 8; u += 32) {
     const int r = u >> 3, ch = u & 7;  // 16 codes = columns 16ch .. 16ch+15
@@ -146,9 +150,9 @@ __device__ __forceinline__ void warp_fp8_rows_to_bf16(const uint8_t* src, int ke
       outv[2 * k + 1] = e4m3x2_to_bf16x2((uint16_t)(w[k] >> 16));
     }
     // bf16 columns 16ch .. 16ch+7 and 16ch+8 .. 16ch+15 -> byte columns 32ch, 32ch+16
-    *reinterpret_cast<uint4*>(dst + sw128_offset(r, ch * 32, rows_out)) =
+    *reinterpret_cast<uint4*>(dst + sw128_offset(dst_row0 + r, ch * 32, rows_out)) =
         make_uint4(outv[0], outv[1], outv[2], outv[3]);
-    *reinterpret_cast<uint4*>(dst + sw128_offset(r, ch * 32 + 16, rows_out)) =
+    *reinterpret_cast<uint4*>(dst + sw128_offset(dst_row0 + r, ch * 32 + 16, rows_out)) =
         make_uint4(outv[4], outv[5], outv[6], outv[7]);
   }
 }

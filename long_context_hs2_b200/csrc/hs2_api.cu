@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "bridge_gemm.cuh"
 #include "full_attn.cuh"
@@ -68,10 +69,6 @@ int sm_count() {
   return n;
 }
 
-hs2_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
-}
-
 // ------------------------------------------------ full-attention plan --
 struct FullPlan {
   bool tc;       // tcgen05 path (D = 128, bf16 cache)
@@ -97,8 +94,9 @@ bool make_full_plan(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt, Full
   pl->groups_per_seq = (T + pl->G - 1) / pl->G;
   pl->n_groups = B * pl->groups_per_seq;
   const int64_t tiles = (L + pl->tile - 1) / pl->tile;
+  // `target` CTAs over the groups, rounded down so that a one-wave grid stays one wave
   auto split = [&](int64_t target, int64_t max_splits, int* n_out, int* keys_out) {
-    int64_t sp = (target + pl->n_groups - 1) / pl->n_groups;
+    int64_t sp = target / pl->n_groups;
     sp = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(sp, tiles), max_splits));
     int64_t per = (L + sp - 1) / sp;
     per = (per + pl->tile - 1) / pl->tile * pl->tile;
@@ -127,22 +125,55 @@ bool make_full_plan(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt, Full
   return true;
 }
 
+// Launches `kernel` on stream s, as clusters of `cluster` CTAs along x when
+// cluster > 1.
+template <typename... KArgs, typename... Args>
+hs2_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                  int cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  int na = 0;
+  if (cluster > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)cluster;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return HS2_ERR_CUDA;
+  }
+  return HS2_OK;
+}
+
 template <typename K>
 bool set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
          cudaSuccess;
 }
 
-hs2_status run_select(const FullAttnParams& fp, const SelectParams& sp, cudaStream_t s) {
-  const long long nc_max = fp.L - fp.window + 1;  // candidates of the last query
-  if (nc_max <= kSelSmemMax) {
-    const int bytes = (int)std::max<long long>(16, nc_max * 4);
-    if (!set_smem(select_topk_kernel<true>, bytes)) return HS2_ERR_CUDA;
-    select_topk_kernel<true><<<(unsigned)(fp.B * fp.T), kSelThreads, bytes, s>>>(sp);
-  } else {
-    select_topk_kernel<false><<<(unsigned)(fp.B * fp.T), kSelThreads, 0, s>>>(sp);
-  }
-  return launch_status();
+hs2_status run_select(const FullAttnParams& fp, SelectParams sp, cudaStream_t s) {
+  // few queries: split each query's candidates over a cluster of up to 8 CTAs
+  const long long rows = (long long)fp.B * fp.T;
+  const int sms = sm_count();
+  int cs = 1;
+  while (cs < 8 && rows * cs * 2 <= sms) cs *= 2;
+  sp.cs = cs;
+  const long long nc_max = std::max<long long>(1, fp.L - fp.window + 1);
+  const long long seg = ((nc_max + cs - 1) / cs + 3) / 4 * 4;
+  const bool smem = seg <= kSelSmemMax;
+  const int bytes = smem ? (int)std::max<long long>(16, seg * 4) : 0;
+  auto k = smem ? select_topk_kernel<true> : select_topk_kernel<false>;
+  if (!set_smem(k, std::max(bytes, 16))) return HS2_ERR_CUDA;
+  return launch(k, dim3((unsigned)(rows * cs)), dim3(kSelThreads), (size_t)bytes, s, cs, sp);
 }
 
 template <int D, bool FP8>
@@ -153,10 +184,11 @@ hs2_status run_full(const CUtensorMap& km, const CUtensorMap& vm, const FullAttn
   auto ks = fp.G == 1 ? attn_score_kernel<D, FP8, 1>
                       : (fp.G == 2 ? attn_score_kernel<D, FP8, 2> : attn_score_kernel<D, FP8, 4>);
   if (!set_smem(kp, SM::kBytes) || !set_smem(ks, SM::kScoreBytes)) return HS2_ERR_CUDA;
-  kp<<<pl.n_groups * pl.n_splits, 160, SM::kBytes, s>>>(km, vm, fp);
-  if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  ks<<<pl.n_groups * pl.score_splits, 160, SM::kScoreBytes, s>>>(km, fp);
-  if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+  hs2_status st = launch(kp, dim3(pl.n_groups * pl.n_splits), dim3(160), SM::kBytes, s, 1, km,
+                         vm, fp);
+  if (st != HS2_OK) return st;
+  st = launch(ks, dim3(pl.n_groups * pl.score_splits), dim3(160), SM::kScoreBytes, s, 1, km, fp);
+  if (st != HS2_OK) return st;
   return run_select(fp, sp, s);
 }
 
@@ -173,10 +205,11 @@ hs2_status run_full_tc(const CUtensorMap& km, const CUtensorMap& vm, const FullA
                                   : (fp.G == 2 ? attn_tc_score_kernel<N, 2>
                                                : attn_tc_score_kernel<N, 4>));
   if (!set_smem(kp, SM::kBytes) || !set_smem(ks, SM::kSBytes)) return HS2_ERR_CUDA;
-  kp<<<pl.n_groups * pl.n_splits, kTcPartialThreads, SM::kBytes, s>>>(km, vm, fp);
-  if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-  ks<<<pl.n_groups * pl.score_splits, kTcThreads, SM::kSBytes, s>>>(km, fp);
-  return launch_status();
+  const hs2_status st = launch(kp, dim3(pl.n_groups * pl.n_splits), dim3(kTcPartialThreads),
+                               SM::kBytes, s, 1, km, vm, fp);
+  if (st != HS2_OK) return st;
+  return launch(ks, dim3(pl.n_groups * pl.score_splits), dim3(kTcThreads), SM::kSBytes, s, 1, km,
+                fp);
 }
 
 template <int MT, int D, bool FP8>
@@ -184,24 +217,8 @@ hs2_status run_sparse(const SparseParams& p, cudaStream_t s) {
   using SM = SparseSmem<MT, D, FP8>;
   auto k = sparse_attn_kernel<MT, D, FP8>;
   if (!set_smem(k, SM::kBytes)) return HS2_ERR_CUDA;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3((unsigned)((long long)p.B * p.T * p.cs));
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = SM::kBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)p.cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, k, p) != cudaSuccess) {
-    cudaGetLastError();
-    return HS2_ERR_CUDA;
-  }
-  return HS2_OK;
+  return launch(k, dim3((unsigned)((long long)p.B * p.T * p.cs)), dim3(128), SM::kBytes, s, p.cs,
+                p);
 }
 
 }  // namespace
@@ -306,6 +323,7 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
   sp.topk = topk;
   sp.window = window;
   sp.slots = topk + window;
+  sp.cs = 1;
 
   cudaStream_t s = (cudaStream_t)stream;
   if (pl.tc) {
@@ -400,8 +418,8 @@ extern "C" hs2_status hs2_bridge_kv(const void* X, int64_t T, int hidden, const 
   if (!set_smem(bridge_gemm_kernel, kBrSmemBytes)) return HS2_ERR_CUDA;
   const long long tiles = (T + kBrBM - 1) / kBrBM * n_layers;
   const int grid = (int)std::min<long long>(tiles, sm_count());
-  bridge_gemm_kernel<<<grid, kBrThreads, kBrSmemBytes, (cudaStream_t)stream>>>(xm, wm, p);
-  return launch_status();
+  return launch(bridge_gemm_kernel, dim3(grid), dim3(kBrThreads), kBrSmemBytes,
+                (cudaStream_t)stream, 1, xm, wm, p);
 }
 
 // ------------------------------------------------------------------------

@@ -1,18 +1,28 @@
 // Token-level top-k selection with the forced recent window.
 //
 // Scores are non-negative fp32 values, so their bit patterns order like the
-// values.  The k-th largest pattern tau is found digit by digit from three
-// histograms (bits [30:20] -- built by attn_score --, [19:9], [8:0]); then one
-// ordered pass keeps every candidate above tau and the first `need` equal to
-// tau (ties go to the lower position), writing positions in ascending order,
-// followed by the window positions i-window+1 .. i.
+// values.  For each query the k-th largest pattern tau is found digit by
+// digit from three histograms (bits [30:20] -- built by the score pass --,
+// then [19:9] and [8:0] over the row); an ordered compaction then keeps every
+// candidate above tau and the first `need` equal to tau (ties go to the lower
+// position), writing positions in ascending order, followed by the window
+// positions i-window+1 .. i.
+//
+// A query's candidates are split into contiguous segments over a thread-block
+// cluster of CS CTAs (CS = 1 when there are many queries).  Each CTA keeps
+// its segment in shared memory when it fits (else reads it from global
+// memory), the digit histograms are summed across the cluster through
+// distributed shared memory, and the compaction offsets each CTA by the
+// survivors of the CTAs before it.  All cross-CTA steps use hardware cluster
+// barriers.
 #pragma once
 
 #include "hs2_common.cuh"
 
 namespace hs2 {
 
-constexpr int kSelThreads = 1024;
+constexpr int kSelThreads = 256;
+constexpr int kSelSmemMax = 48 * 1024;   // candidates of one CTA kept in shared memory
 
 struct SelectParams {
   const float* score;     // [B*T][L]
@@ -21,11 +31,49 @@ struct SelectParams {
   int32_t* n_sel;         // [B*T]
   int T;
   long long L;
-  int topk, window, slots;
+  int topk, window, slots, cs;
 };
 
-// Exclusive prefix sum over the block (1024 threads); returns the total.
-__device__ __forceinline__ int block_exclusive_scan(int v, int& excl, int* warp_tot) {
+__device__ __forceinline__ uint32_t sel_cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void sel_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ uint32_t sel_mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ unsigned ld_dsmem_u32(uint32_t addr) {
+  unsigned v;
+  asm("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void red_dsmem_add_u32(uint32_t addr, unsigned v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint4 ld_dsmem_u32x4(uint32_t addr) {
+  uint4 v;
+  asm("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "r"(addr));
+  return v;
+}
+// Copies rank 0's histogram h (nbins, a multiple of 4) into the local out.
+__device__ __forceinline__ void copy_rank0_hist(const unsigned* h, int nbins, unsigned* out) {
+  const uint32_t base = sel_mapa(smem_u32(h), 0);
+  for (int b = 4 * threadIdx.x; b < nbins; b += 4 * kSelThreads)
+    *reinterpret_cast<uint4*>(out + b) = ld_dsmem_u32x4(base + b * 4);
+}
+
+// Exclusive prefix sum over the CTA (kSelThreads threads); returns the total.
+__device__ __forceinline__ int sel_block_scan(int v, int& excl, int* tmp) {
+  constexpr int W = kSelThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
@@ -33,173 +81,225 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int& excl, int* warp_
     const int y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) warp_tot[warp] = x;
+  if (lane == 31) tmp[warp] = x;
   __syncthreads();
-  if (warp == 0) {
-    int w = warp_tot[lane];
-    int s = w;
+  int before = 0, total = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    warp_tot[32 + lane] = s - w;  // exclusive prefix of warp totals
-    if (lane == 31) warp_tot[64] = s;
+  for (int w = 0; w < W; ++w) {
+    const int t = tmp[w];
+    if (w < warp) before += t;
+    total += t;
   }
-  __syncthreads();
-  excl = x - v + warp_tot[32 + warp];
-  const int total = warp_tot[64];
+  excl = before + x - v;
   __syncthreads();
   return total;
 }
 
-// Given counts hist[0..nbins) and k >= 1, finds the bin `sel` holding the
-// k-th largest element: count(bins > sel) < k <= count(bins >= sel).
-// Writes sel and need = k - count(bins > sel) to out[0], out[1].
-__device__ __forceinline__ void find_kth_bin(const unsigned* hist, int nbins, int k, int* out,
-                                             int* warp_tot) {
+// Bin `sel` holding the k-th largest element of hist[0..nbins) (k >= 1):
+// count(bins > sel) < k <= count(bins >= sel); need = k - count(bins > sel).
+__device__ __forceinline__ void sel_find_bin(const unsigned* hist, int nbins, int k, int* res,
+                                             int* tmp) {
   const int per = (nbins + kSelThreads - 1) / kSelThreads;
-  // thread 0 owns the highest bins
-  const int hi = nbins - threadIdx.x * per;  // exclusive upper bin
+  const int hi = nbins - threadIdx.x * per;  // thread 0 owns the highest bins
   const int lo = max(0, hi - per);
   int local = 0;
-  for (int bb = lo; bb < hi; ++bb) local += (int)hist[bb];
+  for (int b = lo; b < hi; ++b) local += (int)hist[b];
   int excl;
-  block_exclusive_scan(local, excl, warp_tot);
+  sel_block_scan(local, excl, tmp);
   if (excl < k && k <= excl + local) {
     int above = excl;
-    for (int bb = hi - 1; bb >= lo; --bb) {
-      const int cnt = (int)hist[bb];
-      if (above + cnt >= k) {
-        out[0] = bb;
-        out[1] = k - above;
+    for (int b = hi - 1; b >= lo; --b) {
+      const int c = (int)hist[b];
+      if (above + c >= k) {
+        res[0] = b;
+        res[1] = k - above;
         break;
       }
-      above += cnt;
+      above += c;
     }
   }
   __syncthreads();
 }
 
-// SMEM = true: the candidate scores of the row are first copied to dynamic
-// shared memory (rows of at most kSelSmemMax candidates), and every later pass
-// reads them there.  SMEM = false: passes read the row in global memory.
-constexpr int kSelSmemMax = 48 * 1024;
-
 template <bool SMEM>
 __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectParams p) {
-  __shared__ unsigned hist[2048];
-  __shared__ int warp_tot[72];
+  __shared__ unsigned h2[2048];       // this CTA's level-2 histogram
+  __shared__ unsigned h3[512];        // this CTA's level-3 histogram
+  __shared__ unsigned hs[2048];       // cluster sum of the current level
+  __shared__ int tmp[kSelThreads / 32];
   __shared__ int res[2];
-  extern __shared__ unsigned row_s[];
-  const long long row = blockIdx.x;
+  __shared__ int cnt[2];              // this CTA's (count above tau, count equal to tau)
+  __shared__ int wsel[kSelThreads / 32], weq[kSelThreads / 32];
+  extern __shared__ unsigned seg_s[];
+
+  const int cs = p.cs;
+  const uint32_t rank = cs > 1 ? sel_cluster_rank() : 0u;
+  const long long row = blockIdx.x / cs;
   const int t = (int)(row % p.T);
   const long long i = p.L - p.T + t;
   const long long nc = i - p.window + 1;  // candidates 0 .. nc-1
   int32_t* out = p.idx + row * p.slots;
 
   if (nc <= p.topk) {  // every candidate is taken: S = {0 .. i}
-    const long long n = i + 1;
-    for (long long j = threadIdx.x; j < p.slots; j += kSelThreads) out[j] = j < n ? (int32_t)j : -1;
-    if (threadIdx.x == 0) p.n_sel[row] = (int32_t)n;
-    return;
-  }
-  const unsigned* srow_u = reinterpret_cast<const unsigned*>(p.score + row * p.L);
-  if (SMEM) {
-    // 16-byte copies where the row start allows it (p.L % 4 == 0), else words
-    if ((p.L & 3) == 0) {
-      const uint4* g4 = reinterpret_cast<const uint4*>(srow_u);
-      uint4* s4 = reinterpret_cast<uint4*>(row_s);
-      for (long long j = threadIdx.x; j < nc / 4; j += kSelThreads) s4[j] = g4[j];
-      for (long long j = (nc / 4) * 4 + threadIdx.x; j < nc; j += kSelThreads) row_s[j] = srow_u[j];
-    } else {
-      for (long long j = threadIdx.x; j < nc; j += kSelThreads) row_s[j] = srow_u[j];
+    if (rank == 0) {
+      const long long n = i + 1;
+      for (long long j = threadIdx.x; j < p.slots; j += kSelThreads) out[j] = j < n ? (int32_t)j : -1;
+      if (threadIdx.x == 0) p.n_sel[row] = (int32_t)n;
     }
-    __syncthreads();
-    srow_u = row_s;
+    return;  // the same branch for every CTA of the cluster: no cluster barrier follows
   }
+  // this CTA's segment [s0, s1) of the candidates (s0 a multiple of 4)
+  const long long seg = ((nc + cs - 1) / cs + 3) / 4 * 4;
+  const long long s0 = min(nc, (long long)rank * seg), s1 = min(nc, s0 + seg);
+  const unsigned* src = reinterpret_cast<const unsigned*>(p.score + row * p.L) + s0;
+  const int n = (int)(s1 - s0);
+  if (SMEM) {
+    if ((p.L & 3) == 0) {  // 16-byte copies: the row start and s0 are multiples of 4 words
+      const uint4* g4 = reinterpret_cast<const uint4*>(src);
+      uint4* s4 = reinterpret_cast<uint4*>(seg_s);
+      for (int j = threadIdx.x; j < n / 4; j += kSelThreads) s4[j] = g4[j];
+      for (int j = (n / 4) * 4 + threadIdx.x; j < n; j += kSelThreads) seg_s[j] = src[j];
+    } else {
+      for (int j = threadIdx.x; j < n; j += kSelThreads) seg_s[j] = src[j];
+    }
+    src = seg_s;
+  }
+  for (int b = threadIdx.x; b < 2048; b += kSelThreads) h2[b] = 0u;
+  for (int b = threadIdx.x; b < 512; b += kSelThreads) h3[b] = 0u;
+  __syncthreads();
+
   int need = p.topk;
   unsigned prefix = 0;
   if (need > 0) {
-    // level 1: bits [30:20]
-    find_kth_bin(p.hist + row * 2048, 2048, need, res, warp_tot);
+    // level 1: bits [30:20], counted by the score pass
+    sel_find_bin(p.hist + row * 2048, 2048, need, res, tmp);
     prefix = (unsigned)res[0];
     need = res[1];
-    // level 2: bits [19:9] among elements with bits[30:20] == prefix
-    for (int u = threadIdx.x; u < 2048; u += kSelThreads) hist[u] = 0u;
-    __syncthreads();
-    for (long long j = threadIdx.x; j < nc; j += kSelThreads) {
-      const unsigned v = srow_u[j];
-      if ((v >> 20) == prefix) atomicAdd(&hist[(v >> 9) & 2047u], 1u);
+    // level 2: bits [19:9] among elements with bits[30:20] == prefix.  With a
+    // cluster, every CTA counts straight into rank 0's histogram (distributed
+    // shared-memory atomics); after a cluster barrier each CTA copies it.
+    const uint32_t h2_0 = cs > 1 ? sel_mapa(smem_u32(h2), 0) : 0u;
+    if (cs > 1) sel_cluster_sync();  // rank 0's histograms are cleared
+    for (int j = threadIdx.x; j < n; j += kSelThreads) {
+      const unsigned v = src[j];
+      if ((v >> 20) == prefix) {
+        if (cs > 1) red_dsmem_add_u32(h2_0 + ((v >> 9) & 2047u) * 4, 1u);
+        else atomicAdd(&h2[(v >> 9) & 2047u], 1u);
+      }
+    }
+    const unsigned* h = h2;
+    if (cs > 1) {
+      sel_cluster_sync();
+      copy_rank0_hist(h2, 2048, hs);
+      h = hs;
     }
     __syncthreads();
-    find_kth_bin(hist, 2048, need, res, warp_tot);
+    sel_find_bin(h, 2048, need, res, tmp);
     prefix = (prefix << 11) | (unsigned)res[0];
     need = res[1];
     // level 3: bits [8:0] among elements with bits[30:9] == prefix
-    for (int u = threadIdx.x; u < 512; u += kSelThreads) hist[u] = 0u;
-    __syncthreads();
-    for (long long j = threadIdx.x; j < nc; j += kSelThreads) {
-      const unsigned v = srow_u[j];
-      if ((v >> 9) == prefix) atomicAdd(&hist[v & 511u], 1u);
+    const uint32_t h3_0 = cs > 1 ? sel_mapa(smem_u32(h3), 0) : 0u;
+    for (int j = threadIdx.x; j < n; j += kSelThreads) {
+      const unsigned v = src[j];
+      if ((v >> 9) == prefix) {
+        if (cs > 1) red_dsmem_add_u32(h3_0 + (v & 511u) * 4, 1u);
+        else atomicAdd(&h3[v & 511u], 1u);
+      }
+    }
+    h = h3;
+    if (cs > 1) {
+      sel_cluster_sync();
+      copy_rank0_hist(h3, 512, hs);
+      h = hs;
     }
     __syncthreads();
-    find_kth_bin(hist, 512, need, res, warp_tot);
+    sel_find_bin(h, 512, need, res, tmp);
     prefix = (prefix << 9) | (unsigned)res[0];
     need = res[1];
   }
   const unsigned tau = prefix;
-  // Ordered compaction of {v > tau} and the first `need` of {v == tau}.  Warp w
-  // owns the contiguous segment [w*seg, (w+1)*seg) of the candidates: a first
-  // pass counts its survivors (ballots), one block scan orders the warps, and a
-  // second pass writes each warp's survivors at its offset, in index order.
+
+  // Ordered compaction of {v > tau} and the first `need` of {v == tau}: warp w
+  // of the CTA owns the contiguous sub-segment [w*wseg, (w+1)*wseg).
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wseg = (n + kSelThreads / 32 - 1) / (kSelThreads / 32);
+  const int w0 = min(n, warp * wseg), w1 = min(n, w0 + wseg);
+  int n_gt = 0, n_eq = 0;
   if (p.topk > 0) {
-    __shared__ int wsel[32], weq[32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const long long seg = (nc + 31) / 32;
-    const long long s0 = warp * seg, s1 = min(nc, s0 + seg);
-    int n_gt = 0, n_eq = 0;
-    for (long long base = s0; base < s1; base += 32) {
-      const long long j = base + lane;
-      const unsigned v = j < s1 ? srow_u[j] : 0u;
-      n_gt += __popc(__ballot_sync(0xffffffffu, j < s1 && v > tau));
-      n_eq += __popc(__ballot_sync(0xffffffffu, j < s1 && v == tau));
+    for (int base = w0; base < w1; base += 32) {
+      const int j = base + lane;
+      const unsigned v = j < w1 ? src[j] : 0u;
+      n_gt += __popc(__ballot_sync(0xffffffffu, j < w1 && v > tau));
+      n_eq += __popc(__ballot_sync(0xffffffffu, j < w1 && v == tau));
     }
-    if (lane == 0) {
-      wsel[warp] = n_gt;
-      weq[warp] = n_eq;
+  }
+  if (lane == 0) {
+    wsel[warp] = n_gt;
+    weq[warp] = n_eq;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int a = 0, e = 0;
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+      a += wsel[w];
+      e += weq[w];
     }
-    __syncthreads();
-    int gt_before = 0, eq_before = 0;
-    for (int w = 0; w < warp; ++w) {
-      gt_before += wsel[w];
-      eq_before += weq[w];
+    cnt[0] = a;
+    cnt[1] = e;
+  }
+  if (cs > 1) sel_cluster_sync();
+  else __syncthreads();
+  // survivors of the CTAs before this one (lane q of every warp reads rank q's
+  // counts; a warp sum adds them), then of the warps before this one
+  int gt_before = 0, eq_before = 0;
+  if (cs > 1) {
+    const uint32_t caddr = smem_u32(cnt);
+    int g = 0, e = 0;
+    if (lane < (int)rank) {
+      g = (int)ld_dsmem_u32(sel_mapa(caddr, lane));
+      e = (int)ld_dsmem_u32(sel_mapa(caddr + 4, lane));
     }
-    // equal elements taken by this warp: those of rank < need overall
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      g += __shfl_xor_sync(0xffffffffu, g, o);
+      e += __shfl_xor_sync(0xffffffffu, e, o);
+    }
+    gt_before = g;
+    eq_before = e;
+  }
+  for (int w = 0; w < warp; ++w) {
+    gt_before += wsel[w];
+    eq_before += weq[w];
+  }
+  if (p.topk > 0) {
     int pos = gt_before + min(eq_before, need);
     int eq_rank = eq_before;
-    for (long long base = s0; base < s1; base += 32) {
-      const long long j = base + lane;
-      const unsigned v = j < s1 ? srow_u[j] : 0u;
-      const bool gt = j < s1 && v > tau;
-      const bool eq = j < s1 && v == tau;
+    for (int base = w0; base < w1; base += 32) {
+      const int j = base + lane;
+      const unsigned v = j < w1 ? src[j] : 0u;
+      const bool gt = j < w1 && v > tau;
+      const bool eq = j < w1 && v == tau;
       const unsigned eqm = __ballot_sync(0xffffffffu, eq);
       const int my_eq_rank = eq_rank + __popc(eqm & ((1u << lane) - 1u));
       const bool sel = gt || (eq && my_eq_rank < need);
       const unsigned selm = __ballot_sync(0xffffffffu, sel);
       if (sel) {
         const int o = pos + __popc(selm & ((1u << lane) - 1u));
-        if (o < p.topk) out[o] = (int32_t)j;
+        if (o < p.topk) out[o] = (int32_t)(s0 + j);
       }
       pos += __popc(selm);
       eq_rank += __popc(eqm);
     }
-    if (warp == 31 && lane == 0 && pos != p.topk) raise_status(kStatusBadIndex);
+    if (rank == (uint32_t)(cs - 1) && warp == kSelThreads / 32 - 1 && lane == 0 && pos != p.topk)
+      raise_status(kStatusBadIndex);
   }
-  const long long w0 = i - p.window + 1;
-  for (int w = threadIdx.x; w < p.window; w += kSelThreads) out[p.topk + w] = (int32_t)(w0 + w);
-  for (int s = p.topk + p.window + threadIdx.x; s < p.slots; s += kSelThreads) out[s] = -1;
-  if (threadIdx.x == 0) p.n_sel[row] = p.topk + p.window;
+  if (rank == 0) {
+    const long long wstart = i - p.window + 1;
+    for (int w = threadIdx.x; w < p.window; w += kSelThreads) out[p.topk + w] = (int32_t)(wstart + w);
+    for (int s = p.topk + p.window + threadIdx.x; s < p.slots; s += kSelThreads) out[s] = -1;
+    if (threadIdx.x == 0) p.n_sel[row] = p.topk + p.window;
+  }
+  if (cs > 1) sel_cluster_sync();  // no CTA leaves while others may still read its shared memory
 }
 
 }  // namespace hs2

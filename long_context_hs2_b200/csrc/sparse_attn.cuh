@@ -3,13 +3,14 @@
 //
 // One thread-block cluster of CS CTAs per query.  The query's selected slots
 // are cut into 64-slot tiles dealt round-robin to the cluster's CTAs; each CTA
-// first copies (and range-checks) the positions of its slots into shared
-// memory, gathers its tiles' K/V rows with 16-byte cp.async copies into
-// 128B-swizzled shared-memory tiles (a multi-stage ring), runs the warp
-// attention core (warps split every tile's keys 4 ways) and merges its warps.
-// Then every CTA of the cluster merges one slice of the query's H x D output
-// from all CTAs' partials, read through distributed shared memory.  No global
-// scratch is needed.
+// loads (and range-checks) its slots' positions together with the query's
+// n_sel, gathers its tiles' K/V rows with 16-byte cp.async copies into
+// 128B-swizzled shared-memory tiles (a multi-stage ring, all of a decode
+// query's tiles in flight at once), runs the warp attention core (warps split
+// every tile's keys 4 ways) and merges its warps.  Then every CTA of the
+// cluster merges one slice of the query's H x D output from all CTAs'
+// partials, read through distributed shared memory.  No global scratch is
+// needed.
 #pragma once
 
 #include "attn_warp.cuh"
@@ -50,7 +51,7 @@ struct SparseSmem {
   static constexpr int kClBytes = kRowsQ * 8 + kRowsQ * D * 4;
   static constexpr int kPosOff = kClOff + kClBytes;               // positions of the CTA's slots
   static constexpr int kMaxSlots = 4096;
-  static constexpr int kBytes = kPosOff + kMaxSlots * 4 + 1024;
+  static constexpr int kBytes = kPosOff + (kMaxSlots + 64 + 4) * 4 + 1024;
 };
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -123,11 +124,17 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   const int b = (int)(qrow / p.T);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  int n = p.n_sel[qrow];
-  n = max(0, min(n, p.slots));
   const int32_t* sel = p.idx + qrow * p.slots;
-  const int n_tiles_all = (n + kSpTile - 1) / kSpTile;
-  const int my_tiles = n_tiles_all > (int)rank ? (n_tiles_all - (int)rank + cs - 1) / cs : 0;
+  // tiles of this CTA if every slot were used: tile k of the CTA is slot tile rank + k*cs
+  const int tiles_max = (p.slots + kSpTile - 1) / kSpTile;
+  const int my_max = tiles_max > (int)rank ? (tiles_max - (int)rank + cs - 1) / cs : 0;
+  // positions of this CTA's slots, loaded together with n_sel (no dependent round trip)
+  int* nsel_s = pos_all + my_max * kSpTile;
+  if (threadIdx.x == 0) *nsel_s = p.n_sel[qrow];
+  for (int u = threadIdx.x; u < my_max * kSpTile; u += 128) {
+    const int slot = ((int)rank + (u / kSpTile) * cs) * kSpTile + (u % kSpTile);
+    pos_all[u] = slot < p.slots ? sel[slot] : -1;
+  }
 
   // query rows: head h = row (rows >= H are zero)
   {
@@ -142,16 +149,19 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   const float* ksc = FP8 ? p.k_scale + (long long)b * p.L : nullptr;
   const float* vsc = FP8 ? p.v_scale + (long long)b * p.L : nullptr;
 
-  // positions of this CTA's slots: tile k of the CTA is slot tile rank + k*cs
+  __syncthreads();
+  const int n = max(0, min(*nsel_s, p.slots));
+  const int n_tiles_all = (n + kSpTile - 1) / kSpTile;
+  const int my_tiles = n_tiles_all > (int)rank ? (n_tiles_all - (int)rank + cs - 1) / cs : 0;
+  // mask slots past n_sel; range-check the others
   for (int u = threadIdx.x; u < my_tiles * kSpTile; u += 128) {
     const int slot = ((int)rank + (u / kSpTile) * cs) * kSpTile + (u % kSpTile);
-    int ps = -1;
-    if (slot < n) {
-      ps = sel[slot];
-      if (ps < 0 || (long long)ps >= p.L) {
-        raise_status(kStatusBadIndex);
-        ps = -1;
-      }
+    int ps = pos_all[u];
+    if (slot >= n) {
+      ps = -1;
+    } else if (ps < 0 || (long long)ps >= p.L) {
+      raise_status(kStatusBadIndex);
+      ps = -1;
     }
     pos_all[u] = ps;
   }
@@ -173,7 +183,15 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   uint8_t* stg_v = stg_k + 16 * D * 2;
 
   for (int k = 0; k < my_tiles; ++k) {
-    cp_async_wait<SM::kStages - 2>();
+    {  // refill the slot consumed in step k-1 (all threads passed the barrier ending it)
+      const int kn = k + SM::kStages - 1;
+      if (kn < my_tiles)
+        sparse_gather_tile<D, FP8>(p, b, pos_all + kn * kSpTile,
+                                   smem + (kn % SM::kStages) * SM::kStageBytes);
+      else
+        cp_async_commit();
+    }
+    cp_async_wait<SM::kStages - 1>();  // tile k has landed
     __syncthreads();
     const int s = k % SM::kStages;
     uint8_t* stage = smem + s * SM::kStageBytes;
@@ -212,12 +230,6 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
       }
     warp_softmax_pv<MT, D>(st, x, vt, key0, rows, pvs);
     __syncthreads();  // ring slot s is free again
-    const int kn = k + SM::kStages - 1;
-    const int sn = kn % SM::kStages;
-    if (kn < my_tiles)
-      sparse_gather_tile<D, FP8>(p, b, pos_all + kn * kSpTile, smem + sn * SM::kStageBytes);
-    else
-      cp_async_commit();
   }
   cp_async_wait<0>();
   __syncthreads();
