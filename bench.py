@@ -44,7 +44,17 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["hs2", "reference"], default="hs2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bridge", action="store_true")
     return ap.parse_args()
+
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (burst)"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def measured_peaks():
@@ -169,6 +179,57 @@ def run_reference(args, world, rank):
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ KV Bridging --
+def bench_bridge(torch, hs2, args, stream):
+    """Times hs2_bridge_kv on the bridge workload (131072 tokens x 4096 -> 6 layers of
+    K|V, D=128), bf16 and E4M3 outputs, as a tensor-bound roofline beside the decode
+    metric.  Timing inputs are drawn on the device with torch's generator in the
+    workload's distributions (X ~ N(0,1)/64, Wt ~ N(0, 1/4096)); parity of this shape
+    against the oracle is covered by the test suite."""
+    from hs2_synth import WORKLOADS as W
+    wl = W["bridge_131k"]
+    T, hidden, nl, D = wl.T, wl.hidden, wl.n_layers, wl.D
+    g = torch.Generator(device="cuda").manual_seed(wl.seed)
+    x = (torch.randn(T, hidden, device="cuda", generator=g) / 64).to(torch.bfloat16)
+    wt = (torch.randn(nl * 2 * D, hidden, device="cuda", generator=g) / 64).to(torch.bfloat16)
+    out = {}
+    flops = 2.0 * T * hidden * nl * 2 * D
+    peak = measured_tensor_peak()
+    for name, dt in (("bf16", hs2.HS2_KV_BF16), ("fp8", hs2.HS2_KV_FP8_E4M3)):
+        if dt == hs2.HS2_KV_BF16:
+            bufs = [(torch.empty(T, D, dtype=torch.bfloat16, device="cuda"),
+                     torch.empty(T, D, dtype=torch.bfloat16, device="cuda"), None, None)
+                    for _ in range(nl)]
+        else:
+            bufs = [(torch.empty(T, D, dtype=torch.uint8, device="cuda"),
+                     torch.empty(T, D, dtype=torch.uint8, device="cuda"),
+                     torch.empty(T, device="cuda"), torch.empty(T, device="cuda"))
+                    for _ in range(nl)]
+        caches = [hs2.kv_cache(*b) for b in bufs]
+        for _ in range(3):
+            hs2.hs2_bridge_kv(x, T, hidden, wt, nl, D, dt, caches, 0, stream)
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(10)]
+        for a, b in evs:
+            a.record(stream)
+            hs2.hs2_bridge_kv(x, T, hidden, wt, nl, D, dt, caches, 0, stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        st = hs2.hs2_last_device_status()
+        if st != 0:
+            raise RuntimeError("bridge device status: " + hs2.hs2_status_string(st))
+        ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+        tf = flops / (ms * 1e-3) / 1e12
+        out[name] = {"ms": ms, "tflops": tf, "frac": tf / peak[0], "peak": peak[0],
+                     "peak_source": peak[1]}
+        del bufs, caches
+    out["workload"] = "bridge_131k: X [131072 x 4096] bf16, Wt [1536 x 4096] bf16, 6 layers, D=128"
+    out["bound"] = "tensor"
+    out["unit"] = "TFLOP/s"
+    return out
 
 
 # ------------------------------------------------------------------ GPU arm --
@@ -334,6 +395,7 @@ def run_hs2(args, world, rank, local):
         cpu = {"value": rps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": "one full step: %d sequences x 1 query, full attention + selection + "
                          "%d sparse layers (%.1f s)" % (B, wl.n_sparse, dts)}
+    bridge = bench_bridge(torch, hs2, args, stream) if (rank == 0 and not args.no_bridge) else None
     del g_full, g_sparse
     if world > 1:
         dist.barrier()
@@ -370,6 +432,7 @@ def run_hs2(args, world, rank, local):
         "full_ms": full,
         "clocks": clk,
         "cpu_baseline": cpu,
+        "bridge": bridge,
     }
     print(json.dumps(line), flush=True)
 
