@@ -1,5 +1,5 @@
 // Full-attention layer on the 5th-generation tensor cores (tcgen05), for
-// head_dim 128 and a bf16 cache.
+// head_dim 128 and a bf16 or E4M3 cache.
 //
 // MQA: every query row of a group -- N rows = N/H queries x H heads -- reads
 // the same K/V stream.  Each 128-key tile is processed transposed:
@@ -14,9 +14,16 @@
 // no cross-thread max; each thread keeps its keys' partial row sums in a TMEM
 // column block.
 //
-// Warp roles (192 threads): warp 0 issues the TMA loads of the K/V tile ring;
-// warp 1 allocates TMEM and one of its threads issues every tcgen05.mma; warps
-// 2-5 are the softmax warps (one TMEM lane = one key each).
+// Warp roles: warp 0 issues the TMA loads of the K/V tile ring; warp 1
+// allocates TMEM and one of its threads issues every tcgen05.mma; the softmax
+// (or score) warps own one TMEM lane = one key each.
+//
+// E4M3 cache: TMA brings the 128-byte E4M3 rows; converter warps rewrite each
+// K and V tile as f16 (E4M3 -> f16 is exact) in the same 128B-swizzled layout
+// a bf16 tile has, and the MMAs run kind::f16 with f16 operands (Q is staged
+// as f16: exact for bf16 values of magnitude >= 2^-14, and P is written as
+// f16).  The per-token scales need no extra pass: the thread that owns key j
+// multiplies its logits by k_scale[j] and its P values by v_scale[j].
 //   attn_tc_partial : per (group, split): reference max m, sum l and
 //                     un-normalised O of the split.
 //   attn_tc_score   : merges the splits into lse and O, then recomputes S^T per
@@ -30,40 +37,96 @@
 namespace hs2 {
 
 constexpr int kTcKeys = 128;          // keys per tile (M of the score MMA)
-constexpr int kTcTileBytes = kTcKeys * 128 * 2;   // one bf16 K or V tile: 32 KB
+constexpr int kTcTileBytes = kTcKeys * 128 * 2;   // one 16-bit K or V tile: 32 KB
+constexpr int kTcTile8Bytes = kTcKeys * 128;      // one E4M3 K or V tile: 16 KB
 constexpr float kRescaleAbove = 8.f;  // base-2 logits may exceed the reference by this
-constexpr int kTcThreads = 192;
 
-// Shared-memory plan.  Partial kernel: K/V tile ring, Q, P^T (double-buffered
-// for N = 32), per-row reference max / correction / partial maxima and sums.
-template <int N>
+// Shared-memory plan.  Partial kernel: K/V tile ring (16-bit, or E4M3 plus one
+// f16 K and one f16 V tile), Q, P^T (double-buffered for N = 32), per-row
+// reference max / correction / partial maxima and sums.  Score kernel: K ring
+// (plus two f16 K tiles for E4M3), staged (m, l) partials of the group, Q,
+// histograms.
+template <int N, bool FP8>
 struct TcSmem {
-  static constexpr int kStages = N == 32 ? 3 : 2;
+  static constexpr int kStages = FP8 ? (N == 32 ? 4 : 2) : (N == 32 ? 3 : 2);
   static constexpr int kNP = N == 32 ? 2 : 1;            // P^T buffers
-  static constexpr int kStageBytes = 2 * kTcTileBytes;   // K then V
-  static constexpr int kQOff = kStages * kStageBytes;
+  static constexpr int kStageBytes = 2 * (FP8 ? kTcTile8Bytes : kTcTileBytes);  // K then V
+  static constexpr int kK16Off = kStages * kStageBytes;  // E4M3 only: f16 K, then f16 V
+  static constexpr int kQOff = kK16Off + (FP8 ? 2 * kTcTileBytes : 0);
   static constexpr int kQBytes = N * 256;
-  static constexpr int kPOff = kQOff + kQBytes;          // P^T [N rows][128 keys] bf16
+  static constexpr int kPOff = kQOff + kQBytes;          // P^T [N rows][128 keys], 16-bit
   static constexpr int kPBytes = N * 256;
   static constexpr int kMrefOff = kPOff + kNP * kPBytes; // float [N]
   static constexpr int kCorrOff = kMrefOff + N * 4;      // float [N]
   static constexpr int kTmaxOff = kCorrOff + N * 4;      // float [4][N] (also the row sums)
   static constexpr int kBarOff = kTmaxOff + 4 * N * 4;
-  static constexpr int kNumBars = 2 * kStages + 5 + 2 * kNP;
+  static constexpr int kNumBars = 2 * kStages + 9 + 2 * kNP;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kSlotOff + 16 + 1024;
-  // score kernel: K-only ring, staged (m, l) partials of the group, Q, histograms
-  static constexpr int kSStages = N == 32 ? 4 : 3;
-  static constexpr int kSMlOff = kSStages * kTcTileBytes;
+  // score kernel
+  static constexpr int kSStages = (FP8 || N == 32) ? 4 : 3;
+  static constexpr int kSStageBytes = FP8 ? kTcTile8Bytes : kTcTileBytes;
+  static constexpr int kSK16Off = kSStages * kSStageBytes;
+  static constexpr int kSMlOff = kSK16Off + (FP8 ? 2 * kTcTileBytes : 0);
   static constexpr int kSMlBytes = 32 * 1024;            // rows x splits x 8 bytes
   static constexpr int kSQOff = kSMlOff + kSMlBytes;
   static constexpr int kSHistOff = kSQOff + kQBytes;
-  static constexpr int kSHistBytes = (N == 32 ? 4 : 4) * kHistBins * 4;
+  static constexpr int kSHistBytes = 4 * kHistBins * 4;
   static constexpr int kSLseOff = kSHistOff + kSHistBytes;
   static constexpr int kSBarOff = kSLseOff + N * 4;
-  static constexpr int kSSlotOff = kSBarOff + (2 * kSStages + 5) * 8;
+  static constexpr int kSSlotOff = kSBarOff + (2 * kSStages + 9) * 8;
   static constexpr int kSBytes = kSSlotOff + 16 + 1024;
 };
+
+// Rows [row0, row0 + nrows) of an E4M3 tile (TMA layout: 128-byte rows, 16-byte
+// chunks swizzled by row & 7) rewritten as f16 rows of a 128B-swizzled 16-bit
+// tile of 128 rows per column half.  E4M3 -> f16 is exact.
+__device__ __forceinline__ void fp8_rows_to_f16(const uint8_t* src, int row0, int nrows,
+                                                int tid, int nthreads, uint8_t* dst) {
+  for (int u = tid; u < nrows * 8; u += nthreads) {
+    const int r = row0 + (u >> 3), ch = u & 7;  // codes 16ch .. 16ch+15 of row r
+    const uint4 raw = *reinterpret_cast<const uint4*>(src + r * 128 + ((ch ^ (r & 7)) << 4));
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t h[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] & 0xFFFFu), __NV_E4M3);
+      const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] >> 16), __NV_E4M3);
+      h[2 * k] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
+      h[2 * k + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
+    }
+    *reinterpret_cast<uint4*>(dst + sw128_offset(r, ch * 32, kTcKeys)) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(dst + sw128_offset(r, ch * 32 + 16, kTcKeys)) =
+        make_uint4(h[4], h[5], h[6], h[7]);
+  }
+}
+
+// Stages the group's N query rows (row r = query t0 + r/H, head r%H) into a
+// K-major 128B-swizzled 16-bit tile (bf16, or f16 for an E4M3 cache); rows of
+// queries past T are zero.
+template <int N, bool FP8>
+__device__ __forceinline__ void tc_stage_q(const FullAttnParams& p, int b, int t0, uint8_t* qs,
+                                           int tid, int nthreads) {
+  for (int u = tid; u < N * 16; u += nthreads) {
+    const int r = u >> 4, ch = u & 15;
+    const int t = t0 + r / p.H, h = r % p.H;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (t < p.T)
+      v = *reinterpret_cast<const uint4*>(p.q + (((long long)b * p.T + t) * p.H + h) * 128 + ch * 8);
+    if (FP8) {
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(&w[k]);
+        const float2 f = __bfloat1622float2(bb);
+        const __half2 hh = __floats2half2_rn(f.x, f.y);
+        w[k] = *reinterpret_cast<const uint32_t*>(&hh);
+      }
+      v = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    *reinterpret_cast<uint4*>(qs + sw128_offset(r, ch * 16, N)) = v;
+  }
+}
 
 // Barrier, and block-wide OR, over the softmax warps (named barrier 1).
 template <int kThreads>
@@ -94,10 +157,10 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Issues the 8 MMAs of S^T[128 x N] = K_tile . Q^T into TMEM column `d_col`.
-template <int N>
+// Issues the 8 MMAs of S^T[128 x N] = K_tile . Q^T into TMEM at tmem_d.
+template <int N, bool F16>
 __device__ __forceinline__ void tc_issue_qk(uint32_t tmem_d, uint32_t k_addr, uint32_t q_addr) {
-  constexpr uint32_t idesc = tc_idesc_f16(128, N, kTcBF16, false, false);
+  constexpr uint32_t idesc = tc_idesc_f16(128, N, F16 ? kTcF16 : kTcBF16, false, false);
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
     const uint32_t half = ks >> 2, koff = (ks & 3) * 32;
@@ -108,10 +171,10 @@ __device__ __forceinline__ void tc_issue_qk(uint32_t tmem_d, uint32_t k_addr, ui
 
 // Issues the 8 MMAs of O^T[128 x N] (+)= V_tile^T . P, V read MN-major from its
 // TMA tile (d contiguous within a 64-d half, halves 16 KB apart), P^T K-major.
-template <int N>
+template <int N, bool F16>
 __device__ __forceinline__ void tc_issue_pv(uint32_t tmem_d, uint32_t v_addr, uint32_t p_addr,
                                             bool accumulate) {
-  constexpr uint32_t idesc = tc_idesc_f16(128, N, kTcBF16, true, false);
+  constexpr uint32_t idesc = tc_idesc_f16(128, N, F16 ? kTcF16 : kTcBF16, true, false);
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
     const uint32_t half = ks >> 2, koff = (ks & 3) * 32;
@@ -121,22 +184,28 @@ __device__ __forceinline__ void tc_issue_pv(uint32_t tmem_d, uint32_t v_addr, ui
   }
 }
 
-// Partial kernel: warps 0 (TMA), 1 (MMA) and 8 softmax warps 2-9.  Softmax
-// warp w reads TMEM lane quarter w%4 (keys, or d for O^T) and the column half
-// (w-2)/4 of the N rows, so two warps share each scheduler and each thread
-// handles one key x N/2 rows per tile.
-constexpr int kTcPartialThreads = 320;
+// Partial kernel: warps 0 (TMA), 1 (MMA) and 8 softmax warps 2-9 (plus, for
+// an E4M3 cache, K converter warps 10-11 and V converter warps 12-13).
+// Softmax warp w reads TMEM lane quarter w%4 (keys, or d for O^T) and the
+// column half (w-2)/4 of the N rows, so two warps share each scheduler and
+// each thread handles one key x N/2 rows per tile.
 constexpr int kTcSoftmax = 256;
+constexpr int kTcConvert = 64;  // threads per converted tensor (K or V)
+__host__ __device__ constexpr int tc_partial_threads(bool fp8) {
+  return 64 + kTcSoftmax + (fp8 ? 2 * kTcConvert : 0);
+}
+__host__ __device__ constexpr int tc_score_threads(bool fp8) { return fp8 ? 320 : 192; }
 
-template <int N, int G>
-__global__ void __launch_bounds__(kTcPartialThreads, 1)
+template <int N, int G, bool FP8>
+__global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     attn_tc_partial_kernel(const __grid_constant__ CUtensorMap kmap,
                            const __grid_constant__ CUtensorMap vmap, const FullAttnParams p) {
-  using SM = TcSmem<N>;
+  using SM = TcSmem<N, FP8>;
   constexpr int S = SM::kStages;
   constexpr int NP = SM::kNP;
   constexpr int kH = N / G;     // heads per query
   constexpr int NC = N / 2;     // columns per softmax warp
+  constexpr int kTileIn = FP8 ? kTcTile8Bytes : kTcTileBytes;  // one K or V tile as loaded
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   float* m_ref = reinterpret_cast<float*>(smem + SM::kMrefOff);
@@ -149,6 +218,10 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
   uint64_t* p_full = s_empty + 2;    // [NP]
   uint64_t* pv_done = p_full + NP;   // [NP]
   uint64_t* q_ready = pv_done + NP;
+  uint64_t* k16_full = q_ready + 1;  // E4M3 only: converted K / V tile handshakes
+  uint64_t* k16_free = k16_full + 1;
+  uint64_t* v16_full = k16_free + 1;
+  uint64_t* v16_free = v16_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kSlotOff);
 
   const int split = blockIdx.x % p.n_splits;
@@ -178,7 +251,7 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], FP8 ? 2 * kTcConvert / 32 : 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -189,6 +262,10 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(q_ready, kTcSoftmax / 32);
+    mbar_init(k16_full, kTcConvert / 32);
+    mbar_init(k16_free, 1);
+    mbar_init(v16_full, kTcConvert / 32);
+    mbar_init(v16_free, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -214,48 +291,73 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
         uint8_t* st = smem + s * SM::kStageBytes;
         mbar_arrive_expect_tx(&kv_full[s], SM::kStageBytes);
         const int row = (int)((long long)b * p.L + k_lo + (long long)n * kTcKeys);
-        tma_load_2d(st, &kmap, &kv_full[s], 0, row, pol_k);
-        tma_load_2d(st + 16384, &kmap, &kv_full[s], 64, row, pol_k);
-        tma_load_2d(st + kTcTileBytes, &vmap, &kv_full[s], 0, row, pol_v);
-        tma_load_2d(st + kTcTileBytes + 16384, &vmap, &kv_full[s], 64, row, pol_v);
+        if (FP8) {  // 128-byte E4M3 rows: one box per tensor
+          tma_load_2d(st, &kmap, &kv_full[s], 0, row, pol_k);
+          tma_load_2d(st + kTileIn, &vmap, &kv_full[s], 0, row, pol_v);
+        } else {
+          tma_load_2d(st, &kmap, &kv_full[s], 0, row, pol_k);
+          tma_load_2d(st + 16384, &kmap, &kv_full[s], 64, row, pol_k);
+          tma_load_2d(st + kTileIn, &vmap, &kv_full[s], 0, row, pol_v);
+          tma_load_2d(st + kTileIn + 16384, &vmap, &kv_full[s], 64, row, pol_v);
+        }
       }
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------- MMA
     if (lane == 0) {
+      const uint32_t k16_addr = smem_u32(smem + SM::kK16Off);
+      const uint32_t v16_addr = k16_addr + kTcTileBytes;
       bool ok = true;
       auto pv = [&](int m) {
         if (!mbar_wait(&p_full[m % NP], (m / NP) & 1)) return false;
+        if (FP8 && !mbar_wait(v16_full, m & 1)) return false;
         tc_fence_after();
-        tc_issue_pv<N>(tmem + 2 * N, smem_u32(smem + (m % S) * SM::kStageBytes + kTcTileBytes),
-                       p_addr + (m % NP) * SM::kPBytes, m > 0);
+        tc_issue_pv<N, FP8>(tmem + 2 * N,
+                            FP8 ? v16_addr : smem_u32(smem + (m % S) * SM::kStageBytes + kTileIn),
+                            p_addr + (m % NP) * SM::kPBytes, m > 0);
         tc_commit(&pv_done[m % NP]);
-        tc_commit(&kv_empty[m % S]);
+        tc_commit(FP8 ? v16_free : &kv_empty[m % S]);
         return true;
       };
       ok = mbar_wait(q_ready, 0);  // Q staged by the softmax warps
       for (int n = 0; n < n_tiles && ok; ++n) {
         const int s = n % S, bb = n & 1;
-        if (!mbar_wait(&kv_full[s], (n / S) & 1)) break;
+        if (!mbar_wait(FP8 ? k16_full : &kv_full[s], FP8 ? (n & 1) : (n / S) & 1)) break;
         if (n >= 2 && !mbar_wait(&s_empty[bb], ((n - 2) >> 1) & 1)) break;
         tc_fence_after();
-        tc_issue_qk<N>(tmem + bb * N, smem_u32(smem + s * SM::kStageBytes), q_addr);
+        tc_issue_qk<N, FP8>(tmem + bb * N, FP8 ? k16_addr : smem_u32(smem + s * SM::kStageBytes),
+                            q_addr);
         tc_commit(&s_full[bb]);
+        if (FP8) tc_commit(k16_free);
         if (n >= 1) ok = pv(n - 1);
       }
       if (ok) pv(n_tiles - 1);
     }
+  } else if (FP8 && warp >= 2 + kTcSoftmax / 32) {
+    // ----------------------------------------------- E4M3 -> f16 converters
+    const int ct = threadIdx.x - (64 + kTcSoftmax);  // 0..127
+    const bool is_v = ct >= kTcConvert;
+    const int cid = ct % kTcConvert;
+    uint8_t* dst = smem + SM::kK16Off + (is_v ? kTcTileBytes : 0);
+    uint64_t* full16 = is_v ? v16_full : k16_full;
+    uint64_t* free16 = is_v ? v16_free : k16_free;
+    for (int n = 0; n < n_tiles; ++n) {
+      const int s = n % S;
+      if (!mbar_wait(&kv_full[s], (n / S) & 1)) break;
+      if (n >= 1 && !mbar_wait(free16, (n - 1) & 1)) break;  // MMA done with the last tile
+      fp8_rows_to_f16(smem + s * SM::kStageBytes + (is_v ? kTileIn : 0), 0, kTcKeys, cid,
+                      kTcConvert, dst);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&kv_empty[s]);
+        mbar_arrive(full16);
+      }
+    }
   } else {
     // ---------------------------------------------------------- softmax
     // stage Q (read by the tensor cores: fence to the async proxy, then publish)
-    for (int u = threadIdx.x - 64; u < N * 16; u += kTcSoftmax) {
-      const int r = u >> 4, ch = u & 15;
-      const int t = t0 + r / p.H, h = r % p.H;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t < p.T)
-        v = *reinterpret_cast<const uint4*>(p.q + (((long long)b * p.T + t) * p.H + h) * 128 + ch * 8);
-      *reinterpret_cast<uint4*>(smem + SM::kQOff + sw128_offset(r, ch * 16, N)) = v;
-    }
+    tc_stage_q<N, FP8>(p, b, t0, smem + SM::kQOff, threadIdx.x - 64, kTcSoftmax);
     fence_proxy_async_smem();
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(q_ready);
@@ -269,7 +371,6 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
     const int st = threadIdx.x - 64;         // softmax thread 0..255
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const int keyrow = wq * 32 + lane;       // row of S^T (key) / of O^T (d)
-    const float sl = p.scale_log2;
     // P^T store address of (row c0 + c, this key): base + c*128 + xoff[(c0 + c) & 7]
     uint8_t* p_base = smem + SM::kPOff + (keyrow >> 6) * (N * 128) + c0 * 128;
     uint32_t xoff[8];
@@ -286,10 +387,17 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
     }
     for (int n = 0; n < n_tiles; ++n) {
       const int bb = n & 1;
-      failed |= !mbar_wait(&s_full[bb], (n >> 1) & 1);
-      tc_fence_after();
       const long long key0 = k_lo + (long long)n * kTcKeys;
       const long long j = key0 + keyrow;
+      // this key's logit multiplier and P factor (per-token scales of an E4M3 cache)
+      float sl = p.scale_log2, vsc = 1.f;
+      if (FP8) {
+        const bool in = j < k_hi;
+        sl *= in ? p.k_scale[(long long)b * p.L + j] : 0.f;
+        vsc = in ? p.v_scale[(long long)b * p.L + j] : 0.f;
+      }
+      failed |= !mbar_wait(&s_full[bb], (n >> 1) & 1);
+      tc_fence_after();
       // a tile is "full" when every key is in range and causal for every query
       const bool full_tile = key0 + kTcKeys <= k_hi && key0 + kTcKeys - 1 <= p.L - p.T + t0;
       // limit[q]: last key query q of the group may see (in range of this split)
@@ -361,7 +469,8 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
           }
         }
       }
-      // sweep 2: p = 2^(x - m_ref), row sums, P^T (bf16) for the PV product
+      // sweep 2: p = 2^(x - m_ref), row sums, P^T (bf16, or f16 times the
+      // value scale for an E4M3 cache) for the PV product
       uint8_t* pt = p_base + (n % NP) * SM::kPBytes;
 #pragma unroll
       for (int c = 0; c < NC; c += 16) {
@@ -376,8 +485,12 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
           const float mr = m_ref[col];
           const float pr = (ok && mr != kNegInf) ? fast_exp2(x[i] * sl - mr) : 0.f;
           lv[i] += pr;
-          *reinterpret_cast<__nv_bfloat16*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
-              __float2bfloat16_rn(pr);
+          if (FP8)
+            *reinterpret_cast<__half*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
+                __float2half_rn(pr * vsc);
+          else
+            *reinterpret_cast<__nv_bfloat16*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
+                __float2bfloat16_rn(pr);
         }
         tmem_st16(tmem + lane_base + 3 * N + c0 + c, lv);
       }
@@ -429,10 +542,12 @@ __global__ void __launch_bounds__(kTcPartialThreads, 1)
   }
 }
 
-template <int N, int G>
-__global__ void __launch_bounds__(kTcThreads, 1)
+// Score kernel: warps 0 (TMA), 1 (MMA), score warps 2-5 (plus, for an E4M3
+// cache, converter warps 6-9 writing double-buffered f16 K tiles).
+template <int N, int G, bool FP8>
+__global__ void __launch_bounds__(tc_score_threads(FP8), 1)
     attn_tc_score_kernel(const __grid_constant__ CUtensorMap kmap, const FullAttnParams p) {
-  using SM = TcSmem<N>;
+  using SM = TcSmem<N, FP8>;
   constexpr int S = SM::kSStages;
   constexpr int kH = N / G;
   extern __shared__ uint8_t smem_raw[];
@@ -445,6 +560,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* s_full = kv_empty + S;  // [2]
   uint64_t* s_empty = s_full + 2;   // [2]
   uint64_t* q_ready = s_empty + 2;
+  uint64_t* k16_full = q_ready + 1;  // [2], E4M3 only
+  uint64_t* k16_free = k16_full + 2; // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kSSlotOff);
 
   const int split = blockIdx.x % p.score_splits;
@@ -462,11 +579,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], FP8 ? 4 : 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 4);
+      mbar_init(&k16_full[i], 4);
+      mbar_init(&k16_free[i], 1);
     }
     mbar_init(q_ready, 4);
     fence_mbar_init();
@@ -487,11 +606,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int n = 0; n < n_tiles; ++n) {
         const int s = n % S;
         if (n >= S && !mbar_wait(&kv_empty[s], ((n / S) - 1) & 1)) break;
-        uint8_t* st = smem + s * kTcTileBytes;
-        mbar_arrive_expect_tx(&kv_full[s], kTcTileBytes);
+        uint8_t* st = smem + s * SM::kSStageBytes;
+        mbar_arrive_expect_tx(&kv_full[s], SM::kSStageBytes);
         const int row = (int)((long long)b * p.L + k_lo + (long long)n * kTcKeys);
         tma_load_2d(st, &kmap, &kv_full[s], 0, row, pol);
-        tma_load_2d(st + 16384, &kmap, &kv_full[s], 64, row, pol);
+        if (!FP8) tma_load_2d(st + 16384, &kmap, &kv_full[s], 64, row, pol);
       }
     }
   } else if (warp == 1) {
@@ -499,12 +618,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t q_addr = smem_u32(smem + SM::kSQOff);
       for (int n = 0; n < n_tiles; ++n) {
         const int s = n % S, bb = n & 1;
-        if (!mbar_wait(&kv_full[s], (n / S) & 1)) break;
+        if (FP8) {
+          if (!mbar_wait(&k16_full[bb], (n >> 1) & 1)) break;
+        } else if (!mbar_wait(&kv_full[s], (n / S) & 1)) {
+          break;
+        }
         if (n >= 2 && !mbar_wait(&s_empty[bb], ((n - 2) >> 1) & 1)) break;
         tc_fence_after();
-        tc_issue_qk<N>(tmem + bb * N, smem_u32(smem + s * kTcTileBytes), q_addr);
+        tc_issue_qk<N, FP8>(tmem + bb * N,
+                            FP8 ? smem_u32(smem + SM::kSK16Off + bb * kTcTileBytes)
+                                : smem_u32(smem + s * SM::kSStageBytes),
+                            q_addr);
         tc_commit(&s_full[bb]);
-        tc_commit(&kv_empty[s]);
+        tc_commit(FP8 ? &k16_free[bb] : &kv_empty[s]);
+      }
+    }
+  } else if (FP8 && warp >= 6) {
+    // ---- E4M3 -> f16 converters: warp 6 + i converts key rows 32i .. 32i+31
+    const int i = warp - 6;
+    for (int n = 0; n < n_tiles; ++n) {
+      const int s = n % S, bb = n & 1;
+      if (!mbar_wait(&kv_full[s], (n / S) & 1)) break;
+      if (n >= 2 && !mbar_wait(&k16_free[bb], ((n - 2) >> 1) & 1)) break;
+      fp8_rows_to_f16(smem + s * SM::kSStageBytes, 32 * i, 32, lane, 32,
+                      smem + SM::kSK16Off + bb * kTcTileBytes);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&kv_empty[s]);
+        mbar_arrive(&k16_full[bb]);
       }
     }
   } else {
@@ -512,14 +654,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     //      partials, clear the histograms; then lse (base 2) of the group's rows
     const int st = threadIdx.x - 64;
     if (n_tiles > 0) {
-      for (int u = st; u < N * 16; u += 128) {
-        const int r = u >> 4, ch = u & 15;
-        const int t = t0 + r / p.H, h = r % p.H;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (t < p.T)
-          v = *reinterpret_cast<const uint4*>(p.q + (((long long)b * p.T + t) * p.H + h) * 128 + ch * 8);
-        *reinterpret_cast<uint4*>(smem + SM::kSQOff + sw128_offset(r, ch * 16, N)) = v;
-      }
+      tc_stage_q<N, FP8>(p, b, t0, smem + SM::kSQOff, st, 128);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
@@ -548,12 +683,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int wq = warp & 3;
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const int keyrow = wq * 32 + lane;
-    const float sl = p.scale_log2;
     for (int n = 0; n < n_tiles; ++n) {
       const int bb = n & 1;
+      const long long j = k_lo + (long long)n * kTcKeys + keyrow;
+      float sl = p.scale_log2;
+      if (FP8) sl *= j < k_hi ? p.k_scale[(long long)b * p.L + j] : 0.f;
       if (!mbar_wait(&s_full[bb], (n >> 1) & 1)) break;
       tc_fence_after();
-      const long long j = k_lo + (long long)n * kTcKeys + keyrow;
       float acc[G];
 #pragma unroll
       for (int q = 0; q < G; ++q) acc[q] = 0.f;

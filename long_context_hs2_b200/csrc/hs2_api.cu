@@ -71,7 +71,7 @@ int sm_count() {
 
 // ------------------------------------------------ full-attention plan --
 struct FullPlan {
-  bool tc;       // tcgen05 path (D = 128, bf16 cache)
+  bool tc;       // tcgen05 path (D = 128)
   int rows;      // query rows per group (N of the tcgen05 tiles, or 32)
   int tile;      // keys per pipeline tile
   int G, groups_per_seq, n_groups, n_splits, split_keys, score_splits, score_keys;
@@ -87,7 +87,7 @@ bool check_attn_shape(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt) {
 }
 
 bool make_full_plan(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt, FullPlan* pl) {
-  pl->tc = D == 128 && dt == HS2_KV_BF16;
+  pl->tc = D == 128;
   pl->rows = pl->tc && H == 32 && T >= 4 ? 128 : 32;
   pl->tile = pl->tc ? kTcKeys : kTile;
   pl->G = pl->rows / H;
@@ -192,24 +192,25 @@ hs2_status run_full(const CUtensorMap& km, const CUtensorMap& vm, const FullAttn
   return run_select(fp, sp, s);
 }
 
-template <int N>
+template <int N, bool FP8>
 hs2_status run_full_tc(const CUtensorMap& km, const CUtensorMap& vm, const FullAttnParams& fp,
                        const FullPlan& pl, cudaStream_t s) {
-  using SM = TcSmem<N>;
-  auto kp = N == 128 ? attn_tc_partial_kernel<N, 4>
-                     : (fp.G == 1 ? attn_tc_partial_kernel<N, 1>
-                                  : (fp.G == 2 ? attn_tc_partial_kernel<N, 2>
-                                               : attn_tc_partial_kernel<N, 4>));
-  auto ks = N == 128 ? attn_tc_score_kernel<N, 4>
-                     : (fp.G == 1 ? attn_tc_score_kernel<N, 1>
-                                  : (fp.G == 2 ? attn_tc_score_kernel<N, 2>
-                                               : attn_tc_score_kernel<N, 4>));
+  using SM = TcSmem<N, FP8>;
+  static_assert(SM::kBytes <= 232448 && SM::kSBytes <= 232448, "shared memory per CTA");
+  auto kp = N == 128 ? attn_tc_partial_kernel<N, 4, FP8>
+                     : (fp.G == 1 ? attn_tc_partial_kernel<N, 1, FP8>
+                                  : (fp.G == 2 ? attn_tc_partial_kernel<N, 2, FP8>
+                                               : attn_tc_partial_kernel<N, 4, FP8>));
+  auto ks = N == 128 ? attn_tc_score_kernel<N, 4, FP8>
+                     : (fp.G == 1 ? attn_tc_score_kernel<N, 1, FP8>
+                                  : (fp.G == 2 ? attn_tc_score_kernel<N, 2, FP8>
+                                               : attn_tc_score_kernel<N, 4, FP8>));
   if (!set_smem(kp, SM::kBytes) || !set_smem(ks, SM::kSBytes)) return HS2_ERR_CUDA;
-  const hs2_status st = launch(kp, dim3(pl.n_groups * pl.n_splits), dim3(kTcPartialThreads),
-                               SM::kBytes, s, 1, km, vm, fp);
+  const hs2_status st = launch(kp, dim3(pl.n_groups * pl.n_splits),
+                               dim3(tc_partial_threads(FP8)), SM::kBytes, s, 1, km, vm, fp);
   if (st != HS2_OK) return st;
-  return launch(ks, dim3(pl.n_groups * pl.score_splits), dim3(kTcThreads), SM::kSBytes, s, 1, km,
-                fp);
+  return launch(ks, dim3(pl.n_groups * pl.score_splits), dim3(tc_score_threads(FP8)), SM::kSBytes,
+                s, 1, km, fp);
 }
 
 template <int MT, int D, bool FP8>
@@ -328,7 +329,10 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
   cudaStream_t s = (cudaStream_t)stream;
   if (pl.tc) {
     const hs2_status st =
-        pl.rows == 128 ? run_full_tc<128>(km, vm, fp, pl, s) : run_full_tc<32>(km, vm, fp, pl, s);
+        fp8 ? (pl.rows == 128 ? run_full_tc<128, true>(km, vm, fp, pl, s)
+                              : run_full_tc<32, true>(km, vm, fp, pl, s))
+            : (pl.rows == 128 ? run_full_tc<128, false>(km, vm, fp, pl, s)
+                              : run_full_tc<32, false>(km, vm, fp, pl, s));
     if (st != HS2_OK) return st;
     return run_select(fp, sp, s);
   }
