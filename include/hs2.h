@@ -206,6 +206,22 @@ HS2_API hs2_status hs2_last_device_status(hs2_stream_t stream);
 /* Static English description of a status code. */
 HS2_API const char* hs2_status_string(hs2_status status);
 
+/*
+ * Optional timing of the dominant launch of hs2_full_attn_select (and of
+ * hs2_full_attn_select_noalloc): its partial-attention kernel, the one pass
+ * over the whole K/V cache.  While a pair is set, each of those calls made on
+ * this host thread records `begin_event` on its stream just before that
+ * kernel and `end_event` just after it, so that cudaEventElapsedTime of the
+ * pair is the kernel's device time.  Inside stream capture the records become
+ * external event nodes of the graph (cudaEventRecordExternal), recorded at
+ * every replay.
+ *   begin_event, end_event: cudaEvent_t handles owned by the caller, created
+ *     with timing enabled; both null clears the pair (the default).
+ * Returns HS2_ERR_INVALID_ARG when exactly one of the two is null.  Nothing is
+ * enqueued by this call.
+ */
+HS2_API hs2_status hs2_set_stage_events(void* begin_event, void* end_event);
+
 /* Library ABI version: 100 * major + minor. */
 HS2_API int hs2_version(void);
 

@@ -25,7 +25,7 @@ _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error",
 
 EXPORTED = ("hs2_bridge_kv", "hs2_full_attn_select_workspace", "hs2_full_attn_select",
             "hs2_full_attn_select_noalloc", "hs2_sparse_attn", "hs2_last_device_status",
-            "hs2_status_string", "hs2_version")
+            "hs2_status_string", "hs2_version", "hs2_set_stage_events")
 
 # Size of the scratch area built into the library for hs2_full_attn_select_noalloc.
 HS2_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -71,6 +71,8 @@ def load_library(path: str = LIB_PATH):
     lib.hs2_full_attn_select_noalloc.restype = i32
     lib.hs2_full_attn_select_noalloc.argtypes = [P, KV, i32, i32, i64, i32, i32, ctypes.c_float,
                                                  i32, i32, i32, P, P, P, P, P]
+    lib.hs2_set_stage_events.restype = i32
+    lib.hs2_set_stage_events.argtypes = [P, P]
     lib.hs2_sparse_attn.restype = i32
     lib.hs2_sparse_attn.argtypes = [P, KV, i32, i32, i64, i32, i32, ctypes.c_float, P, P, i32, i32,
                                     P, P]
@@ -154,3 +156,14 @@ def hs2_sparse_attn(Q, kv: hs2_kv_cache, B, T, L, H, D, scale, idx, n_sel, slots
     _check("hs2_sparse_attn", load_library().hs2_sparse_attn(
         _ptr(Q), ctypes.byref(kv), int(B), int(T), int(L), int(H), int(D), float(scale),
         _ptr(idx), _ptr(n_sel), int(slots), int(dt), _ptr(O), _stream(stream)))
+
+
+def hs2_set_stage_events(begin=None, end=None):
+    """Sets (or, with no arguments, clears) the events that this thread's
+    full-attention calls record around their partial-attention kernel.
+    `begin`/`end` are torch.cuda.Event objects (timing enabled) or raw handles."""
+    def handle(e):
+        if e is None or isinstance(e, int):
+            return e
+        return e.cuda_event
+    _check("hs2_set_stage_events", load_library().hs2_set_stage_events(handle(begin), handle(end)))

@@ -69,6 +69,21 @@ int sm_count() {
   return n;
 }
 
+// ------------------------------------------- optional stage timing --
+thread_local cudaEvent_t t_stage_begin = nullptr, t_stage_end = nullptr;
+
+// Records the caller's stage event (if any) on s; an external event node when
+// s is being captured into a graph.
+cudaError_t stage_mark(cudaStream_t s, bool begin) {
+  cudaEvent_t ev = begin ? t_stage_begin : t_stage_end;
+  if (!ev) return cudaSuccess;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return cudaErrorUnknown;
+  return cs == cudaStreamCaptureStatusActive
+             ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+             : cudaEventRecord(ev, s);
+}
+
 // ------------------------------------------------ full-attention plan --
 struct FullPlan {
   bool tc;       // tcgen05 path (D = 128)
@@ -184,9 +199,11 @@ hs2_status run_full(const CUtensorMap& km, const CUtensorMap& vm, const FullAttn
   auto ks = fp.G == 1 ? attn_score_kernel<D, FP8, 1>
                       : (fp.G == 2 ? attn_score_kernel<D, FP8, 2> : attn_score_kernel<D, FP8, 4>);
   if (!set_smem(kp, SM::kBytes) || !set_smem(ks, SM::kScoreBytes)) return HS2_ERR_CUDA;
+  if (stage_mark(s, true) != cudaSuccess) return HS2_ERR_CUDA;
   hs2_status st = launch(kp, dim3(pl.n_groups * pl.n_splits), dim3(160), SM::kBytes, s, 1, km,
                          vm, fp);
   if (st != HS2_OK) return st;
+  if (stage_mark(s, false) != cudaSuccess) return HS2_ERR_CUDA;
   st = launch(ks, dim3(pl.n_groups * pl.score_splits), dim3(160), SM::kScoreBytes, s, 1, km, fp);
   if (st != HS2_OK) return st;
   return run_select(fp, sp, s);
@@ -206,9 +223,11 @@ hs2_status run_full_tc(const CUtensorMap& km, const CUtensorMap& vm, const FullA
                                   : (fp.G == 2 ? attn_tc_score_kernel<N, 2, FP8>
                                                : attn_tc_score_kernel<N, 4, FP8>));
   if (!set_smem(kp, SM::kBytes) || !set_smem(ks, SM::kSBytes)) return HS2_ERR_CUDA;
+  if (stage_mark(s, true) != cudaSuccess) return HS2_ERR_CUDA;
   const hs2_status st = launch(kp, dim3(pl.n_groups * pl.n_splits),
                                dim3(tc_partial_threads(FP8)), SM::kBytes, s, 1, km, vm, fp);
   if (st != HS2_OK) return st;
+  if (stage_mark(s, false) != cudaSuccess) return HS2_ERR_CUDA;
   return launch(ks, dim3(pl.n_groups * pl.score_splits), dim3(tc_score_threads(FP8)), SM::kSBytes,
                 s, 1, km, fp);
 }
@@ -226,7 +245,14 @@ hs2_status run_sparse(const SparseParams& p, cudaStream_t s) {
 
 extern "C" {
 
-int hs2_version(void) { return 100; }
+int hs2_version(void) { return 101; }
+
+hs2_status hs2_set_stage_events(void* begin_event, void* end_event) {
+  if ((begin_event == nullptr) != (end_event == nullptr)) return HS2_ERR_INVALID_ARG;
+  t_stage_begin = static_cast<cudaEvent_t>(begin_event);
+  t_stage_end = static_cast<cudaEvent_t>(end_event);
+  return HS2_OK;
+}
 
 const char* hs2_status_string(hs2_status st) {
   switch (st) {

@@ -92,6 +92,12 @@ def test_sparse_attn_rejects_bad_arguments(lib):
     assert f(16, ctypes.byref(kv8), 1, 1, 64, 32, 64, 0.1, 16, 16, 8, 1, 16, None) == 2  # fp8 needs D=128
 
 
+def test_stage_events_pairing(lib):
+    assert lib.hs2_set_stage_events(ctypes.c_void_p(16), None) == 1
+    assert lib.hs2_set_stage_events(None, ctypes.c_void_p(16)) == 1
+    assert lib.hs2_set_stage_events(None, None) == 0
+
+
 def test_product_path_does_not_import_oracle():
     pkg = os.path.join(ROOT, "long_context_hs2_b200")
     for dirpath, _, files in os.walk(pkg):
