@@ -233,8 +233,8 @@ def bench_bridge(torch, hs2, args, stream):
 
 
 # ------------------------------------------------------------------ GPU arm --
-PARTIAL_PROFILE = os.path.join(ROOT, "profiles", "attn_tc_partial_decode_bf16_32k.md")
-KERNEL_SOURCES = ("attn_tc.cuh", "tc_common.cuh", "hs2_common.cuh", "full_attn.cuh")
+PARTIAL_PROFILE = os.path.join(ROOT, "profiles", "attn_tc_fused_decode_bf16_32k.md")
+KERNEL_SOURCES = ("attn_tc.cuh", "tc_common.cuh", "hs2_common.cuh", "full_attn.cuh", "select.cuh")
 
 
 def kernel_source_hash():
@@ -290,11 +290,26 @@ def run_hs2(args, world, rank, local):
     qs = [up(q, torch.bfloat16) for q in [inp.q] + inp.q_sparse]
     ws_bytes = hs2.hs2_full_attn_select_workspace(B, T, L, H, D, wl.topk, wl.window, dt)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
-    outs = [torch.empty(B, T, H, D, dtype=torch.float32, device="cuda") for _ in qs]
-    idx = torch.empty(B, T, slots, dtype=torch.int32, device="cuda")
-    nsel = torch.empty(B, T, dtype=torch.int32, device="cuda")
+    # the step's inputs (all layers' queries) and results (outputs, indices,
+    # counts) each live in one device buffer, so that the end-to-end steps move
+    # them with one host-to-device and one device-to-host copy
+    n_q = B * T * H * D
+    q_all = torch.empty(len(qs) * n_q, dtype=torch.bfloat16, device="cuda")
+    d_q = [q_all[i * n_q:(i + 1) * n_q].view(B, T, H, D) for i in range(len(qs))]
+    n_out = len(qs) * n_q + B * T * slots + B * T
+    out_all = torch.empty(n_out, dtype=torch.float32, device="cuda")
+    outs = [out_all[i * n_q:(i + 1) * n_q].view(B, T, H, D) for i in range(len(qs))]
+    o_idx = len(qs) * n_q
+    idx = out_all[o_idx:o_idx + B * T * slots].view(torch.int32).view(B, T, slots)
+    nsel = out_all[o_idx + B * T * slots:].view(torch.int32).view(B, T)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
+
+    def l2_flush():
+        # write a buffer larger than L2, then read it back so that no dirty
+        # lines of the flush are left to be written back inside the next step
+        flush.zero_()
+        flush.view(torch.int32).sum()
 
     def step(q_list):
         hs2.hs2_full_attn_select(q_list[0], kv, B, T, L, H, D, wl.scale, wl.topk, wl.window, dt,
@@ -313,7 +328,7 @@ def run_hs2(args, world, rank, local):
                                 outs[1 + s])
 
     for _ in range(args.warmup):
-        flush.zero_()
+        l2_flush()
         step(qs)
     torch.cuda.synchronize()
     st = hs2.hs2_last_device_status()
@@ -322,9 +337,8 @@ def run_hs2(args, world, rank, local):
 
     # The block's launches are captured into CUDA graphs (full layer; the three
     # sparse layers) and replayed every step, as a decode loop would.  Each
-    # timed step has its own full-layer graph whose partial-attention kernel
+    # timed step has its own full-layer graph whose fused attention kernel
     # (the dominant launch) is bracketed by that step's pair of stage events.
-    d_q = [torch.empty_like(q) for q in qs]
     for dq, q in zip(d_q, qs):
         dq.copy_(q)
     stage_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -344,7 +358,7 @@ def run_hs2(args, world, rank, local):
     with torch.cuda.graph(g_sparse):
         sparse_layers(d_q)
     for i in range(max(args.warmup, args.steps)):
-        flush.zero_()
+        l2_flush()
         g_full[i % args.steps].replay()
         g_sparse.replay()
     torch.cuda.synchronize()
@@ -359,7 +373,7 @@ def run_hs2(args, world, rank, local):
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
-        flush.zero_()
+        l2_flush()
         e0, e1, e2 = ev[i]
         e0.record(stream)
         g_full[i].replay()
@@ -381,31 +395,24 @@ def run_hs2(args, world, rank, local):
         raise RuntimeError("device status after timing: " + hs2.hs2_status_string(st))
 
     # ---- end to end: pinned host queries in, outputs back, every step
-    h_q = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for q in qs]
-    for hq, q in zip(h_q, qs):
-        hq.copy_(q.cpu())
-    h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-    h_idx = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
-    h_ns = torch.empty(nsel.shape, dtype=nsel.dtype, pin_memory=True)
-    h2d = sum(q.numel() * q.element_size() for q in qs)
-    d2h = sum(o.numel() * o.element_size() for o in outs) + idx.numel() * 4 + nsel.numel() * 4
+    h_q = torch.empty(q_all.shape, dtype=q_all.dtype, pin_memory=True)
+    h_q.copy_(q_all.cpu())
+    h_out = torch.empty(out_all.shape, dtype=out_all.dtype, pin_memory=True)
+    h2d = q_all.numel() * q_all.element_size()
+    d2h = out_all.numel() * out_all.element_size()
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
-        flush.zero_()
+        l2_flush()
         a, c = e2e_ev[i]
         a.record(stream)
-        for dq, hq in zip(d_q, h_q):
-            dq.copy_(hq, non_blocking=True)
+        q_all.copy_(h_q, non_blocking=True)
         g_full[i].replay()
         g_sparse.replay()
-        for ho, o in zip(h_out, outs):
-            ho.copy_(o, non_blocking=True)
-        h_idx.copy_(idx, non_blocking=True)
-        h_ns.copy_(nsel, non_blocking=True)
+        h_out.copy_(out_all, non_blocking=True)
         c.record(stream)
     torch.cuda.synchronize()
     e2e_ms = [a.elapsed_time(c) for a, c in e2e_ev]
@@ -424,7 +431,7 @@ def run_hs2(args, world, rank, local):
     partial = agg(partial_ms)
     e2e = agg(e2e_ms)
     peak, peak_kind = measured_peaks()
-    # algorithmic bytes of the dominant kernel (partial attention: one pass over
+    # algorithmic bytes of the dominant kernel (the fused attention pass: one pass over
     # K and V, plus the queries) and of one sparse layer (the selected K/V rows,
     # queries, outputs, indices)
     partial_bytes = 2 * B * L * D * 2 + B * T * H * D * 2
@@ -461,13 +468,16 @@ def run_hs2(args, world, rank, local):
         "config": {"workload": WORKLOAD, "B": B, "T": T, "L": L, "H": H, "D": D,
                    "kv": "bf16", "topk": wl.topk, "window": wl.window,
                    "sparse_layers": wl.n_sparse, "parallelism": "replicas (dp%d)" % world,
-                   "l2": "flushed before each step (512 MB write)"},
+                   "l2": "flushed before each step (512 MB write, then read back)"},
         "e2e": {"value": tokens / (e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": (3 + wl.n_sparse) * args.steps,
+        # per step: the fused full-attention kernel (partials, score and
+        # selection in one launch for this shape) and one per sparse layer
+        "gpu_launches": (1 + wl.n_sparse) * args.steps,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "attn_tc_partial_kernel<32,1,bf16> (one pass over K/V)",
+                     "kernel": "attn_tc_fused_kernel<32,1,bf16> (partials over K/V, score pass, "
+                               "selection; algorithmic bytes: K and V once, and the queries)",
                      "algorithmic_bytes": partial_bytes, "ms": partial,
                      "peak_source": peak_kind},
         "sparse_layer": {"ms": sparse, "achieved_gbs": sparse_bytes / (sparse * 1e-3) / 1e9,

@@ -208,11 +208,13 @@ HS2_API const char* hs2_status_string(hs2_status status);
 
 /*
  * Optional timing of the dominant launch of hs2_full_attn_select (and of
- * hs2_full_attn_select_noalloc): its partial-attention kernel, the one pass
- * over the whole K/V cache.  While a pair is set, each of those calls made on
- * this host thread records `begin_event` on its stream just before that
- * kernel and `end_event` just after it, so that cudaEventElapsedTime of the
- * pair is the kernel's device time.  Inside stream capture the records become
+ * hs2_full_attn_select_noalloc): the kernel that makes the one pass over the
+ * whole K/V cache (for head_dim 128 and 32 query rows per group, the fused
+ * kernel that also computes the scores and, when they fit, the selection).
+ * While a pair is set, each of those calls made on this host thread records
+ * `begin_event` on its stream just before that kernel and `end_event` just
+ * after it, so that cudaEventElapsedTime of the pair is the kernel's device
+ * time.  Inside stream capture the records become
  * external event nodes of the graph (cudaEventRecordExternal), recorded at
  * every replay.
  *   begin_event, end_event: cudaEvent_t handles owned by the caller, created

@@ -32,6 +32,7 @@
 #pragma once
 
 #include "full_attn.cuh"
+#include "select.cuh"
 #include "tc_common.cuh"
 
 namespace hs2 {
@@ -62,7 +63,18 @@ struct TcSmem {
   static constexpr int kBarOff = kTmaxOff + 4 * N * 4;
   static constexpr int kNumBars = 2 * kStages + 9 + 2 * kNP;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kSlotOff + 16 + 1024;
+  static constexpr int kBar2Off = kSlotOff + 16;         // fused kernel: score-pass barriers
+  static constexpr int kNumBars2 = 16;
+  static constexpr int kBytes = kBar2Off + kNumBars2 * 8 + 1024;
+  // fused kernel: the score pass reuses the partial pass's tile ring for its
+  // K ring, the group's (m, l) partials and the histograms; the fused
+  // selection then uses it for the row's candidate scores and its counters
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kS2Stages = 4;
+  static constexpr int kS2TileBytes = FP8 ? kTcTile8Bytes : kTcTileBytes;
+  static constexpr int kS2MlOff = kS2Stages * kS2TileBytes;  // float2 [N][splits], <= 32 KB
+  static constexpr int kS2HistOff = kS2MlOff + 32 * 1024;    // unsigned [G][2048], <= 32 KB
+  static constexpr bool kFusable = kS2HistOff + 32 * 1024 <= kRingBytes;
   // score kernel
   static constexpr int kSStages = (FP8 || N == 32) ? 4 : 3;
   static constexpr int kSStageBytes = FP8 ? kTcTile8Bytes : kTcTileBytes;
@@ -196,18 +208,58 @@ __host__ __device__ constexpr int tc_partial_threads(bool fp8) {
 }
 __host__ __device__ constexpr int tc_score_threads(bool fp8) { return fp8 ? 320 : 192; }
 
+// Barrier initialisation and per-row state of the partial pass (all threads;
+// a block barrier must follow before the body runs).
+template <int N, bool FP8>
+__device__ __forceinline__ void tc_partial_setup(uint8_t* smem) {
+  using SM = TcSmem<N, FP8>;
+  constexpr int S = SM::kStages;
+  constexpr int NP = SM::kNP;
+  float* m_ref = reinterpret_cast<float*>(smem + SM::kMrefOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
+  if (threadIdx.x < N) m_ref[threadIdx.x] = kNegInf;
+  if (threadIdx.x == 0) {
+    uint64_t* kv_full = bars;
+    uint64_t* kv_empty = kv_full + S;
+    uint64_t* s_full = kv_empty + S;
+    uint64_t* s_empty = s_full + 2;
+    uint64_t* p_full = s_empty + 2;
+    uint64_t* pv_done = p_full + NP;
+    uint64_t* q_ready = pv_done + NP;
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], FP8 ? 2 * kTcConvert / 32 : 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], kTcSoftmax / 32);
+    }
+    for (int i = 0; i < NP; ++i) {
+      mbar_init(&p_full[i], kTcSoftmax / 32);
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(q_ready, kTcSoftmax / 32);
+    mbar_init(q_ready + 1, kTcConvert / 32);  // k16_full
+    mbar_init(q_ready + 2, 1);                // k16_free
+    mbar_init(q_ready + 3, kTcConvert / 32);  // v16_full
+    mbar_init(q_ready + 4, 1);                // v16_free
+    fence_mbar_init();
+  }
+}
+
+// The partial pass of one (group, split) work item: every role's work, with
+// the barriers of tc_partial_setup initialised and 4N TMEM columns at `tmem`.
+// Returns in every thread once its role is done (no trailing barrier).
 template <int N, int G, bool FP8>
-__global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
-    attn_tc_partial_kernel(const __grid_constant__ CUtensorMap kmap,
-                           const __grid_constant__ CUtensorMap vmap, const FullAttnParams p) {
+__device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                                const FullAttnParams& p, uint8_t* smem,
+                                                uint32_t tmem) {
   using SM = TcSmem<N, FP8>;
   constexpr int S = SM::kStages;
   constexpr int NP = SM::kNP;
   constexpr int kH = N / G;     // heads per query
   constexpr int NC = N / 2;     // columns per softmax warp
   constexpr int kTileIn = FP8 ? kTcTile8Bytes : kTcTileBytes;  // one K or V tile as loaded
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
   float* m_ref = reinterpret_cast<float*>(smem + SM::kMrefOff);
   float* corr = reinterpret_cast<float*>(smem + SM::kCorrOff);
   float* tmax = reinterpret_cast<float*>(smem + SM::kTmaxOff);
@@ -222,7 +274,6 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   uint64_t* k16_free = k16_full + 1;
   uint64_t* v16_full = k16_free + 1;
   uint64_t* v16_free = v16_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kSlotOff);
 
   const int split = blockIdx.x % p.n_splits;
   const int grp = blockIdx.x / p.n_splits;
@@ -246,36 +297,6 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     return;
   }
   const int n_tiles = (int)((k_hi - k_lo + kTcKeys - 1) / kTcKeys);
-
-  if (threadIdx.x < N) m_ref[threadIdx.x] = kNegInf;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], FP8 ? 2 * kTcConvert / 32 : 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], kTcSoftmax / 32);
-    }
-    for (int i = 0; i < NP; ++i) {
-      mbar_init(&p_full[i], kTcSoftmax / 32);
-      mbar_init(&pv_done[i], 1);
-    }
-    mbar_init(q_ready, kTcSoftmax / 32);
-    mbar_init(k16_full, kTcConvert / 32);
-    mbar_init(k16_free, 1);
-    mbar_init(v16_full, kTcConvert / 32);
-    mbar_init(v16_free, 1);
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, 4 * N);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
   const uint32_t q_addr = smem_u32(smem + SM::kQOff);
   const uint32_t p_addr = smem_u32(smem + SM::kPOff);
 
@@ -284,7 +305,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     if (lane == 0) {
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      const uint64_t pol_k = policy_evict_last(), pol_v = policy_evict_first();
+      const uint64_t pol_k = policy_evict_normal(), pol_v = policy_evict_first();
       for (int n = 0; n < n_tiles; ++n) {
         const int s = n % S;
         if (n >= S && !mbar_wait(&kv_empty[s], ((n / S) - 1) & 1)) break;
@@ -535,6 +556,460 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     }
     tc_fence_before();
   }
+}
+
+template <int N, int G, bool FP8>
+__global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
+    attn_tc_partial_kernel(const __grid_constant__ CUtensorMap kmap,
+                           const __grid_constant__ CUtensorMap vmap, const FullAttnParams p) {
+  using SM = TcSmem<N, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kSlotOff);
+  tc_partial_setup<N, FP8>(smem);
+  if (threadIdx.x / 32 == 1) {
+    tmem_alloc(tmem_slot, 4 * N);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  tc_partial_body<N, G, FP8>(kmap, vmap, p, smem, tmem);
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x / 32 == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 4 * N);
+  }
+}
+
+
+// Arrival at a group-wide barrier of CTAs through a global counter (zeroed
+// before the launch), then a bounded wait until `target` CTAs have arrived.
+// Whole CTA.  The CTAs of a group must be co-resident (cooperative launch).
+__device__ __forceinline__ void group_arrive_wait(unsigned* ctr, unsigned target) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1u);
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t it = 0;; ++it) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+      if (v >= target) break;
+      if (it >= (1u << 24) || ((it & 15u) == 15u && globaltimer() - t0 > kWaitLimitNs)) {
+        raise_status(kStatusTimeout);
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+  }
+  __syncthreads();
+}
+
+// Fused decode pass: the partial pass of this CTA's (group, split), then --
+// once every split of the group has its partials -- the score pass over the
+// same split's keys (its K tiles are still in L2) while four warps merge this
+// split's share of the group's output rows, then (fuse_select) the selection
+// of the group's rows by all of the group's CTAs together: each keeps its
+// split's candidate scores in shared memory, adds them to the level-2 and
+// level-3 digit histograms in global memory between group barriers, and
+// writes its survivors at the offset the lower splits' counts give.  Without
+// fuse_select a separate selection kernel follows.
+template <int N, int G, bool FP8>
+__global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
+    attn_tc_fused_kernel(const __grid_constant__ CUtensorMap kmap,
+                         const __grid_constant__ CUtensorMap vmap, const FullAttnParams p) {
+  using SM = TcSmem<N, FP8>;
+  static_assert(SM::kFusable, "score pass does not fit the tile ring");
+  constexpr int kThreads = tc_partial_threads(FP8);
+  constexpr int S2 = SM::kS2Stages;
+  constexpr int kH = N / G;
+  constexpr int W = kThreads / 32;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int s_res[2], s_tmp[32], s_prefix[4], s_need[4], s_base[2];
+  __shared__ int s_wg[4][16], s_we[4][16];
+  uint8_t* smem = align1024(smem_raw);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kSlotOff);
+  uint64_t* kv2_full = reinterpret_cast<uint64_t*>(smem + SM::kBar2Off);
+  uint64_t* kv2_empty = kv2_full + S2;
+  uint64_t* s2_full = kv2_empty + S2;  // [2]
+  uint64_t* s2_empty = s2_full + 2;    // [2]
+  uint64_t* k2_full = s2_empty + 2;    // [2], E4M3 only
+  uint64_t* k2_free = k2_full + 2;     // [2]
+
+  tc_partial_setup<N, FP8>(smem);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S2; ++s) {
+      mbar_init(&kv2_full[s], 1);
+      mbar_init(&kv2_empty[s], FP8 ? 4 : 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s2_full[i], 1);
+      mbar_init(&s2_empty[i], 4);
+      mbar_init(&k2_full[i], 4);
+      mbar_init(&k2_free[i], 1);
+    }
+    fence_mbar_init();
+  }
+  if (threadIdx.x / 32 == 1) {
+    tmem_alloc(tmem_slot, 4 * N);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // ------------------------------------------------------------ partials
+  tc_partial_body<N, G, FP8>(kmap, vmap, p, smem, tmem);
+
+  const int ns = p.n_splits;
+  const int split = blockIdx.x % ns;
+  const int grp = blockIdx.x / ns;
+  const int b = grp / p.groups_per_seq;
+  const int t0 = (grp % p.groups_per_seq) * G;
+  const int t_last = min(p.T, t0 + G) - 1;
+  const long long i_last = p.L - p.T + t_last;
+  const long long k_lo = (long long)split * p.split_keys;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  unsigned* gsync = p.grp_sync + 8 * grp;
+  if (p.fuse_select && split == 0)  // the group's level-2/3 counters start at zero
+    for (int q = 0; q < G && t0 + q < p.T; ++q) {
+      const long long row = (long long)b * p.T + t0 + q;
+      for (int u = threadIdx.x; u < 2048; u += kThreads) p.hist2[row * 2048 + u] = 0u;
+      for (int u = threadIdx.x; u < 512; u += kThreads) p.hist3[row * 512 + u] = 0u;
+    }
+  tc_fence_before();
+  group_arrive_wait(gsync, (unsigned)ns);  // the group's partials are out
+  tc_fence_after();
+
+  // --------------------------------------------------------- score pass
+  const long long k2_hi = min(k_lo + (long long)p.split_keys, i_last - p.window + 1);
+  const int n2 = k_lo < k2_hi ? (int)((k2_hi - k_lo + kTcKeys - 1) / kTcKeys) : 0;
+  float2* ml_s = reinterpret_cast<float2*>(smem + SM::kS2MlOff);  // [N][ns]
+  unsigned* hist_s = reinterpret_cast<unsigned*>(smem + SM::kS2HistOff);
+  float* lse2_s = reinterpret_cast<float*>(smem + SM::kCorrOff);
+  uint8_t* k16 = smem + SM::kK16Off;  // E4M3: two f16 K tiles
+  // fuse_select: this split's candidate scores of row q at seg[q * split_keys + (j - k_lo)]
+  float* seg = reinterpret_cast<float*>(smem + SM::kPOff);
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      for (int n = 0; n < n2; ++n) {
+        const int s = n % S2;
+        if (n >= S2 && !mbar_wait(&kv2_empty[s], ((n / S2) - 1) & 1)) break;
+        uint8_t* st = smem + s * SM::kS2TileBytes;
+        mbar_arrive_expect_tx(&kv2_full[s], SM::kS2TileBytes);
+        const int row = (int)((long long)b * p.L + k_lo + (long long)n * kTcKeys);
+        tma_load_2d(st, &kmap, &kv2_full[s], 0, row, pol);
+        if (!FP8) tma_load_2d(st + 16384, &kmap, &kv2_full[s], 64, row, pol);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(smem + SM::kQOff);
+      for (int n = 0; n < n2; ++n) {
+        const int s = n % S2, bb = n & 1;
+        if (FP8) {
+          if (!mbar_wait(&k2_full[bb], (n >> 1) & 1)) break;
+        } else if (!mbar_wait(&kv2_full[s], (n / S2) & 1)) {
+          break;
+        }
+        if (n >= 2 && !mbar_wait(&s2_empty[bb], ((n - 2) >> 1) & 1)) break;
+        tc_fence_after();
+        tc_issue_qk<N, FP8>(tmem + bb * N,
+                            FP8 ? smem_u32(k16 + bb * kTcTileBytes)
+                                : smem_u32(smem + s * SM::kS2TileBytes),
+                            q_addr);
+        tc_commit(&s2_full[bb]);
+        tc_commit(FP8 ? &k2_free[bb] : &kv2_empty[s]);
+      }
+    }
+  } else if (FP8 && warp >= 2 + kTcSoftmax / 32) {
+    // E4M3 -> f16: converter warp 10 + i takes key rows 32i .. 32i+31 of a tile
+    const int i = warp - (2 + kTcSoftmax / 32);
+    if (i < 4)
+      for (int n = 0; n < n2; ++n) {
+        const int s = n % S2, bb = n & 1;
+        if (!mbar_wait(&kv2_full[s], (n / S2) & 1)) break;
+        if (n >= 2 && !mbar_wait(&k2_free[bb], ((n - 2) >> 1) & 1)) break;
+        fp8_rows_to_f16(smem + s * SM::kS2TileBytes, 32 * i, 32, lane, 32, k16 + bb * kTcTileBytes);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&kv2_empty[s]);
+          mbar_arrive(&k2_full[bb]);
+        }
+      }
+  } else {
+    // warps 2-9: the group's (m, l) partials and lse (base 2) of its rows
+    const int st = threadIdx.x - 64;
+    const float2* ml_g = p.part_ml + (long long)grp * ns * N;
+    for (int u = st; u < N * ns; u += kTcSoftmax) {
+      const int sp = u / N, r = u % N;
+      ml_s[r * ns + sp] = __ldcg(ml_g + (long long)sp * N + r);
+    }
+    softmax_sync<kTcSoftmax>();
+    for (int r = st; r < N; r += kTcSoftmax) {
+      float M = kNegInf;
+      for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, ml_s[r * ns + sp].x);
+      float lt = 0.f;
+      if (M != kNegInf)
+        for (int sp = 0; sp < ns; ++sp) {
+          const float2 v = ml_s[r * ns + sp];
+          lt += v.x == kNegInf ? 0.f : v.y * fast_exp2(v.x - M);
+        }
+      lse2_s[r] = M + log2f(lt);
+    }
+    softmax_sync<kTcSoftmax>();
+    if (warp < 6) {
+      // ---- score warps 2-5: one key (TMEM lane) each per tile
+      const int sc = threadIdx.x - 64;
+      for (int u = sc; u < G * kHistBins; u += 128) hist_s[u] = 0u;
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+      const int wq = warp & 3;
+      const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+      const int keyrow = wq * 32 + lane;
+      for (int n = 0; n < n2; ++n) {
+        const int bb = n & 1;
+        const long long j = k_lo + (long long)n * kTcKeys + keyrow;
+        float sl = p.scale_log2;
+        if (FP8) sl *= j < k2_hi ? p.k_scale[(long long)b * p.L + j] : 0.f;
+        if (!mbar_wait(&s2_full[bb], (n >> 1) & 1)) break;
+        tc_fence_after();
+        float acc[G];
+#pragma unroll
+        for (int q = 0; q < G; ++q) acc[q] = 0.f;
+#pragma unroll
+        for (int c = 0; c < N / 32; ++c) {
+          float x[32];
+          tmem_ld32(tmem + lane_base + bb * N + 32 * c, x);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            acc[(32 * c + i) / kH] += fast_exp2(x[i] * sl - lse2_s[32 * c + i]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s2_empty[bb]);
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+          const int t = t0 + q;
+          if (t < p.T && j <= p.L - p.T + t - p.window) {
+            p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
+            if (p.fuse_select) seg[q * p.split_keys + (int)(j - k_lo)] = acc[q];
+            atomicAdd(&hist_s[q * kHistBins + (__float_as_uint(acc[q]) >> kHistShift)], 1u);
+          }
+        }
+      }
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+      for (int u = sc; u < G * kHistBins; u += 128) {
+        const unsigned cnt = hist_s[u];
+        const int t = t0 + u / kHistBins;
+        if (cnt && t < p.T)
+          atomicAdd(&p.hist[((long long)b * p.T + t) * kHistBins + (u % kHistBins)], cnt);
+      }
+    } else {
+      // ---- merge warps 6-9: output row r of the group is merged by the CTA of
+      //      split r mod ns; thread d owns element d
+      const int d = threadIdx.x - 192;
+      for (int r = split; r < N; r += ns) {
+        const int t = t0 + r / kH;
+        if (t >= p.T) continue;
+        const float l2 = lse2_s[r];
+        const long long li = ((long long)b * p.T + t) * p.H + r % kH;
+        if (d == 0) {
+          p.lse[li] = l2 * 0.69314718055994531f;
+          if (p.lse_out) p.lse_out[li] = l2 * 0.69314718055994531f;
+        }
+        const float* po = p.part_o + ((long long)grp * ns * N + r) * 128 + d;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int sp = 0; sp < ns; ++sp) {
+          const float2 v = ml_s[r * ns + sp];
+          const float f = (v.x == kNegInf) ? 0.f : fast_exp2(v.x - l2);
+          acc += f * __ldcg(po + (long long)sp * N * 128);
+        }
+        p.o[li * 128 + d] = acc;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+
+  // ------------------------------------------ selection (whole group)
+  // Three digit levels of the k-th largest score pattern tau, as in
+  // select_topk_kernel: bits [30:20] (the score pass's histogram), [19:9] and
+  // [8:0]; then the ordered compaction of {v > tau} and the first `need` of
+  // {v == tau}.  Every CTA of the group takes every barrier.
+  if (p.fuse_select) {
+    const unsigned* segu = reinterpret_cast<const unsigned*>(seg);
+    auto row_of = [&](int q) { return (long long)b * p.T + t0 + q; };
+    auto nc_of = [&](int q) { return p.L - p.T + t0 + q - p.window + 1; };
+    auto active = [&](int q) { return t0 + q < p.T && nc_of(q) > p.topk && p.topk > 0; };
+    auto nseg_of = [&](int q) {
+      return (int)max(0LL, min((long long)p.split_keys, nc_of(q) - k_lo));
+    };
+    group_arrive_wait(gsync + 1, (unsigned)ns);  // level-1 counts complete
+#pragma unroll 1
+    for (int q = 0; q < G; ++q)
+      if (active(q)) {
+        sel_find_bin_global<kThreads, 2048>(p.hist + row_of(q) * kHistBins, p.topk, s_res, s_tmp);
+        if (threadIdx.x == 0) {
+          s_prefix[q] = s_res[0];
+          s_need[q] = s_res[1];
+        }
+      }
+    __syncthreads();
+#pragma unroll 1
+    for (int q = 0; q < G; ++q)
+      if (active(q)) {
+        const unsigned pre = (unsigned)s_prefix[q];
+        unsigned* h = p.hist2 + row_of(q) * 2048;
+        const int n = nseg_of(q);
+        for (int u = threadIdx.x; u < n; u += kThreads) {
+          const unsigned v = segu[q * p.split_keys + u];
+          if ((v >> 20) == pre) atomicAdd(h + ((v >> 9) & 2047u), 1u);
+        }
+      }
+    group_arrive_wait(gsync + 2, (unsigned)ns);  // level-2 counts complete
+#pragma unroll 1
+    for (int q = 0; q < G; ++q)
+      if (active(q)) {
+        sel_find_bin_global<kThreads, 2048>(p.hist2 + row_of(q) * 2048, s_need[q], s_res, s_tmp);
+        if (threadIdx.x == 0) {
+          s_prefix[q] = (s_prefix[q] << 11) | s_res[0];
+          s_need[q] = s_res[1];
+        }
+      }
+    __syncthreads();
+#pragma unroll 1
+    for (int q = 0; q < G; ++q)
+      if (active(q)) {
+        const unsigned pre = (unsigned)s_prefix[q];
+        unsigned* h = p.hist3 + row_of(q) * 512;
+        const int n = nseg_of(q);
+        for (int u = threadIdx.x; u < n; u += kThreads) {
+          const unsigned v = segu[q * p.split_keys + u];
+          if ((v >> 9) == pre) atomicAdd(h + (v & 511u), 1u);
+        }
+      }
+    group_arrive_wait(gsync + 3, (unsigned)ns);  // level-3 counts complete
+#pragma unroll 1
+    for (int q = 0; q < G; ++q)
+      if (active(q)) {
+        sel_find_bin_global<kThreads, 512>(p.hist3 + row_of(q) * 512, s_need[q], s_res, s_tmp);
+        if (threadIdx.x == 0) {
+          s_prefix[q] = (s_prefix[q] << 9) | s_res[0];
+          s_need[q] = s_res[1];
+        }
+      }
+    __syncthreads();
+    // counts above / equal to tau of each warp's contiguous part of this split
+#pragma unroll 1
+    for (int q = 0; q < G; ++q)
+      if (active(q)) {
+        const unsigned tau = (unsigned)s_prefix[q];
+        const int n = nseg_of(q);
+        const int wseg = (n + W - 1) / W;
+        const int w0 = min(n, warp * wseg), w1 = min(n, w0 + wseg);
+        int n_gt = 0, n_eq = 0;
+        for (int base = w0; base < w1; base += 32) {
+          const int u = base + lane;
+          const unsigned v = u < w1 ? segu[q * p.split_keys + u] : 0u;
+          n_gt += __popc(__ballot_sync(0xffffffffu, u < w1 && v > tau));
+          n_eq += __popc(__ballot_sync(0xffffffffu, u < w1 && v == tau));
+        }
+        if (lane == 0) {
+          s_wg[q][warp] = n_gt;
+          s_we[q][warp] = n_eq;
+        }
+      }
+    __syncthreads();
+    if (threadIdx.x < G && active(threadIdx.x)) {
+      int g = 0, e = 0;
+      for (int w = 0; w < W; ++w) {
+        g += s_wg[threadIdx.x][w];
+        e += s_we[threadIdx.x][w];
+      }
+      p.sel_cnt[row_of(threadIdx.x) * ns + split] = make_int2(g, e);
+    }
+    group_arrive_wait(gsync + 4, (unsigned)ns);  // every split's counts are out
+#pragma unroll 1
+    for (int q = 0; q < G; ++q)
+      if (active(q)) {
+        if (warp == 0) {  // survivors of the lower splits
+          int g = 0, e = 0;
+          for (int sp = lane; sp < split; sp += 32) {
+            const int2 c = __ldcg(p.sel_cnt + row_of(q) * ns + sp);
+            g += c.x;
+            e += c.y;
+          }
+#pragma unroll
+          for (int o = 16; o; o >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, o);
+            e += __shfl_xor_sync(0xffffffffu, e, o);
+          }
+          if (lane == 0) {
+            s_base[0] = g;
+            s_base[1] = e;
+          }
+        }
+        __syncthreads();
+        const unsigned tau = (unsigned)s_prefix[q];
+        const int need = s_need[q];
+        int gt_before = s_base[0], eq_before = s_base[1];
+        for (int w = 0; w < warp; ++w) {
+          gt_before += s_wg[q][w];
+          eq_before += s_we[q][w];
+        }
+        const int n = nseg_of(q);
+        const int wseg = (n + W - 1) / W;
+        const int w0 = min(n, warp * wseg), w1 = min(n, w0 + wseg);
+        int32_t* out = p.idx + row_of(q) * p.slots;
+        int pos = gt_before + min(eq_before, need);
+        int eq_rank = eq_before;
+        for (int base = w0; base < w1; base += 32) {
+          const int u = base + lane;
+          const unsigned v = u < w1 ? segu[q * p.split_keys + u] : 0u;
+          const bool gt = u < w1 && v > tau;
+          const bool eq = u < w1 && v == tau;
+          const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+          const int my_eq_rank = eq_rank + __popc(eqm & ((1u << lane) - 1u));
+          const bool sel = gt || (eq && my_eq_rank < need);
+          const unsigned selm = __ballot_sync(0xffffffffu, sel);
+          if (sel) {
+            const int o = pos + __popc(selm & ((1u << lane) - 1u));
+            if (o < p.topk) out[o] = (int32_t)(k_lo + u);
+          }
+          pos += __popc(selm);
+          eq_rank += __popc(eqm);
+        }
+        if (split == ns - 1 && warp == W - 1 && lane == 0 && pos != p.topk)
+          raise_status(kStatusBadIndex);
+        __syncthreads();  // s_base is rewritten for the next row
+      }
+    if (split == 0)  // window, padding and count; or every position when all are taken
+      for (int q = 0; q < G && t0 + q < p.T; ++q) {
+        const long long i = p.L - p.T + t0 + q;
+        int32_t* out = p.idx + row_of(q) * p.slots;
+        if (nc_of(q) <= p.topk) {
+          for (int j = threadIdx.x; j < p.slots; j += kThreads) out[j] = j <= i ? (int32_t)j : -1;
+          if (threadIdx.x == 0) p.n_sel[row_of(q)] = (int32_t)(i + 1);
+        } else {
+          const long long wstart = i - p.window + 1;
+          for (int w = threadIdx.x; w < p.window; w += kThreads)
+            out[p.topk + w] = (int32_t)(wstart + w);
+          for (int j = p.topk + p.window + threadIdx.x; j < p.slots; j += kThreads) out[j] = -1;
+          if (threadIdx.x == 0) p.n_sel[row_of(q)] = p.topk + p.window;
+        }
+      }
+  }
+  tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

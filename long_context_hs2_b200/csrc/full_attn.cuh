@@ -41,6 +41,15 @@ struct FullAttnParams {
   int G, groups_per_seq, n_splits, split_keys, window;
   int score_splits, score_keys;  // split of the score pass (finer than the partials')
   float scale_log2;
+  // fused tcgen05 pass only: per-group arrival counters (zeroed before the
+  // launch), and the selection outputs when the selection is fused too
+  unsigned* grp_sync;            // [groups][8]
+  unsigned* hist2;               // [B*T][2048] level-2 counts (fused selection)
+  unsigned* hist3;               // [B*T][512]  level-3 counts
+  int2* sel_cnt;                 // [B*T][splits] (above, equal to) the threshold per split
+  int32_t* idx;                  // [B*T][slots]
+  int32_t* n_sel;                // [B*T]
+  int topk, slots, fuse_select;
 };
 
 template <int D, bool FP8>
@@ -154,7 +163,7 @@ __global__ void __launch_bounds__(160) attn_partial_kernel(const __grid_constant
     if (lane == 0) {
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      const uint64_t pol_k = policy_evict_last(), pol_v = policy_evict_first();
+      const uint64_t pol_k = policy_evict_normal(), pol_v = policy_evict_first();
       for (int n = 0; n < n_tiles; ++n) {
         const int s = n % SM::kStages;
         if (n >= SM::kStages && !mbar_wait(&empty[s], ((n / SM::kStages) - 1) & 1)) break;

@@ -87,10 +87,12 @@ cudaError_t stage_mark(cudaStream_t s, bool begin) {
 // ------------------------------------------------ full-attention plan --
 struct FullPlan {
   bool tc;       // tcgen05 path (D = 128)
+  bool fused;    // one fused tcgen05 kernel (partials, score and selection) for N = 32
   int rows;      // query rows per group (N of the tcgen05 tiles, or 32)
   int tile;      // keys per pipeline tile
   int G, groups_per_seq, n_groups, n_splits, split_keys, score_splits, score_keys;
-  size_t off_part_o, off_part_ml, off_lse, off_hist, off_score, total;
+  size_t off_part_o, off_part_ml, off_lse, off_hist, off_score, off_sync, off_hist2, off_hist3,
+      off_cnt, total;
 };
 
 bool check_attn_shape(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt) {
@@ -104,6 +106,7 @@ bool check_attn_shape(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt) {
 bool make_full_plan(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt, FullPlan* pl) {
   pl->tc = D == 128;
   pl->rows = pl->tc && H == 32 && T >= 4 ? 128 : 32;
+  pl->fused = pl->tc && pl->rows == 32;
   pl->tile = pl->tc ? kTcKeys : kTile;
   pl->G = pl->rows / H;
   pl->groups_per_seq = (T + pl->G - 1) / pl->G;
@@ -136,28 +139,43 @@ bool make_full_plan(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt, Full
   off = align_up(off + (size_t)B * T * kHistBins * 4, 256);
   pl->off_score = off;
   off = align_up(off + (size_t)B * T * (size_t)L * 4, 256);
+  pl->off_sync = pl->off_hist2 = pl->off_hist3 = pl->off_cnt = off;
+  if (pl->fused) {
+    off = align_up(off + (size_t)pl->n_groups * 8 * 4, 256);
+    pl->off_hist2 = off;
+    off = align_up(off + (size_t)B * T * 2048 * 4, 256);
+    pl->off_hist3 = off;
+    off = align_up(off + (size_t)B * T * 512 * 4, 256);
+    pl->off_cnt = off;
+    off = align_up(off + (size_t)B * T * pl->n_splits * 8, 256);
+  }
   pl->total = off;
   return true;
 }
 
 // Launches `kernel` on stream s, as clusters of `cluster` CTAs along x when
-// cluster > 1.
+// cluster > 1, and as a cooperative grid (all CTAs co-resident, or the launch
+// fails) when coop.
 template <typename... KArgs, typename... Args>
-hs2_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                  int cluster, Args&&... args) {
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+hs2_status launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     int cluster, bool coop, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   int na = 0;
   if (cluster > 1) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
     attr[na].val.clusterDim.x = (unsigned)cluster;
     attr[na].val.clusterDim.y = 1;
     attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (coop) {
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na].val.cooperative = 1;
     ++na;
   }
   cfg.attrs = attr;
@@ -167,6 +185,12 @@ hs2_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, 
     return HS2_ERR_CUDA;
   }
   return HS2_OK;
+}
+
+template <typename... KArgs, typename... Args>
+hs2_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                  int cluster, Args&&... args) {
+  return launch_ex(kernel, grid, block, smem, s, cluster, false, std::forward<Args>(args)...);
 }
 
 template <typename K>
@@ -230,6 +254,34 @@ hs2_status run_full_tc(const CUtensorMap& km, const CUtensorMap& vm, const FullA
   if (stage_mark(s, false) != cudaSuccess) return HS2_ERR_CUDA;
   return launch(ks, dim3(pl.n_groups * pl.score_splits), dim3(tc_score_threads(FP8)), SM::kSBytes,
                 s, 1, km, fp);
+}
+
+// The fused tcgen05 pass (N = 32): arrival counters cleared, then one
+// cooperative launch (the CTAs of a group wait for one another); the
+// selection runs inside it when a row's candidates fit its shared memory,
+// else as the selection kernel after it.
+template <bool FP8>
+hs2_status run_fused_tc(const CUtensorMap& km, const CUtensorMap& vm, FullAttnParams fp,
+                        const FullPlan& pl, const SelectParams& sp, cudaStream_t s) {
+  using SM = TcSmem<32, FP8>;
+  static_assert(SM::kBytes <= 232448, "shared memory per CTA");
+  // the selection is fused when a split's candidate scores of the group's
+  // rows fit the P^T buffers (shared memory free after the partial pass)
+  fp.fuse_select = (long long)fp.G * fp.split_keys * 4 <= SM::kNP * SM::kPBytes;
+  auto kf = fp.G == 1 ? attn_tc_fused_kernel<32, 1, FP8>
+                      : (fp.G == 2 ? attn_tc_fused_kernel<32, 2, FP8>
+                                   : attn_tc_fused_kernel<32, 4, FP8>);
+  if (!set_smem(kf, SM::kBytes)) return HS2_ERR_CUDA;
+  if (cudaMemsetAsync(fp.grp_sync, 0, (size_t)pl.n_groups * 8 * 4, s) != cudaSuccess) {
+    cudaGetLastError();
+    return HS2_ERR_CUDA;
+  }
+  if (stage_mark(s, true) != cudaSuccess) return HS2_ERR_CUDA;
+  const hs2_status st = launch_ex(kf, dim3(pl.n_groups * pl.n_splits), dim3(tc_partial_threads(FP8)),
+                                  SM::kBytes, s, 1, pl.n_splits > 1, km, vm, fp);
+  if (st != HS2_OK) return st;
+  if (stage_mark(s, false) != cudaSuccess) return HS2_ERR_CUDA;
+  return fp.fuse_select ? HS2_OK : run_select(fp, sp, s);
 }
 
 template <int MT, int D, bool FP8>
@@ -352,7 +404,19 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
   sp.slots = topk + window;
   sp.cs = 1;
 
+  fp.grp_sync = reinterpret_cast<unsigned*>(ws + pl.off_sync);
+  fp.hist2 = reinterpret_cast<unsigned*>(ws + pl.off_hist2);
+  fp.hist3 = reinterpret_cast<unsigned*>(ws + pl.off_hist3);
+  fp.sel_cnt = reinterpret_cast<int2*>(ws + pl.off_cnt);
+  fp.idx = idx;
+  fp.n_sel = n_sel;
+  fp.topk = topk;
+  fp.slots = topk + window;
+  fp.fuse_select = 0;
+
   cudaStream_t s = (cudaStream_t)stream;
+  if (pl.fused)
+    return fp8 ? run_fused_tc<true>(km, vm, fp, pl, sp, s) : run_fused_tc<false>(km, vm, fp, pl, sp, s);
   if (pl.tc) {
     const hs2_status st =
         fp8 ? (pl.rows == 128 ? run_full_tc<128, true>(km, vm, fp, pl, s)

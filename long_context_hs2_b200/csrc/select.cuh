@@ -71,9 +71,10 @@ __device__ __forceinline__ void copy_rank0_hist(const unsigned* h, int nbins, un
     *reinterpret_cast<uint4*>(out + b) = ld_dsmem_u32x4(base + b * 4);
 }
 
-// Exclusive prefix sum over the CTA (kSelThreads threads); returns the total.
+// Exclusive prefix sum over the CTA (kThreads threads); returns the total.
+template <int kThreads = kSelThreads>
 __device__ __forceinline__ int sel_block_scan(int v, int& excl, int* tmp) {
-  constexpr int W = kSelThreads / 32;
+  constexpr int W = kThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
@@ -97,25 +98,64 @@ __device__ __forceinline__ int sel_block_scan(int v, int& excl, int* tmp) {
 
 // Bin `sel` holding the k-th largest element of hist[0..nbins) (k >= 1):
 // count(bins > sel) < k <= count(bins >= sel); need = k - count(bins > sel).
+// With kGlobal, hist is global memory that may have been written earlier in
+// the same grid, and is read through L2 (ld.global.cg); else shared memory.
+template <int kThreads = kSelThreads, bool kGlobal = false>
 __device__ __forceinline__ void sel_find_bin(const unsigned* hist, int nbins, int k, int* res,
                                              int* tmp) {
-  const int per = (nbins + kSelThreads - 1) / kSelThreads;
-  const int hi = nbins - threadIdx.x * per;  // thread 0 owns the highest bins
+  const int per = (nbins + kThreads - 1) / kThreads;
+  const int hi = max(0, nbins - (int)threadIdx.x * per);  // thread 0 owns the highest bins
   const int lo = max(0, hi - per);
   int local = 0;
-  for (int b = lo; b < hi; ++b) local += (int)hist[b];
+  for (int b = lo; b < hi; ++b) local += (int)(kGlobal ? __ldcg(hist + b) : hist[b]);
   int excl;
-  sel_block_scan(local, excl, tmp);
+  sel_block_scan<kThreads>(local, excl, tmp);
   if (excl < k && k <= excl + local) {
     int above = excl;
     for (int b = hi - 1; b >= lo; --b) {
-      const int c = (int)hist[b];
+      const int c = (int)(kGlobal ? __ldcg(hist + b) : hist[b]);
       if (above + c >= k) {
         res[0] = b;
         res[1] = k - above;
         break;
       }
       above += c;
+    }
+  }
+  __syncthreads();
+}
+
+// Bin holding the k-th largest element of a global histogram of NB bins
+// (k >= 1), read through L2 (it may have been written earlier in the same
+// grid): each thread loads its bins into registers with independent loads,
+// then a block scan finds the owner.  res[0] = bin, res[1] = k - count(bins
+// above it).  Whole CTA (kThreads threads).
+template <int kThreads, int NB>
+__device__ __forceinline__ void sel_find_bin_global(const unsigned* hist, int k, int* res,
+                                                    int* tmp) {
+  constexpr int PER = (NB + kThreads - 1) / kThreads;
+  const int hi = NB - (int)threadIdx.x * PER;  // thread 0 owns the highest bins
+  unsigned c[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    const int bin = hi - 1 - e;
+    c[e] = bin >= 0 && hi > 0 ? __ldcg(hist + bin) : 0u;
+  }
+  int local = 0;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) local += (int)c[e];
+  int excl;
+  sel_block_scan<kThreads>(local, excl, tmp);
+  if (excl < k && k <= excl + local) {
+    int above = excl;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      if (above + (int)c[e] >= k) {
+        res[0] = hi - 1 - e;
+        res[1] = k - above;
+        break;
+      }
+      above += (int)c[e];
     }
   }
   __syncthreads();
@@ -172,7 +212,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
   unsigned prefix = 0;
   if (need > 0) {
     // level 1: bits [30:20], counted by the score pass
-    sel_find_bin(p.hist + row * 2048, 2048, need, res, tmp);
+    sel_find_bin<kSelThreads, true>(p.hist + row * 2048, 2048, need, res, tmp);
     prefix = (unsigned)res[0];
     need = res[1];
     // level 2: bits [19:9] among elements with bits[30:20] == prefix.  With a
