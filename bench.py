@@ -309,7 +309,7 @@ def run_hs2(args, world, rank, local):
         # write a buffer larger than L2, then read it back so that no dirty
         # lines of the flush are left to be written back inside the next step
         flush.zero_()
-        flush.view(torch.int32).sum()
+        flush.view(torch.int64).amax()
 
     def step(q_list):
         hs2.hs2_full_attn_select(q_list[0], kv, B, T, L, H, D, wl.scale, wl.topk, wl.window, dt,

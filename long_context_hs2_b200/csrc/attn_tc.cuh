@@ -75,6 +75,8 @@ struct TcSmem {
   static constexpr int kS2MlOff = kS2Stages * kS2TileBytes;  // float2 [N][splits], <= 32 KB
   static constexpr int kS2HistOff = kS2MlOff + 32 * 1024;    // unsigned [G][2048], <= 32 KB
   static constexpr bool kFusable = kS2HistOff + 32 * 1024 <= kRingBytes;
+  static constexpr int kSelWorkOff = kRingBytes - 16 * 1024;  // counters, list offsets
+  static constexpr int kSelCap = kSelWorkOff / 4;             // list entries held in smem
   // score kernel
   static constexpr int kSStages = (FP8 || N == 32) ? 4 : 3;
   static constexpr int kSStageBytes = FP8 ? kTcTile8Bytes : kTcTileBytes;
@@ -613,11 +615,9 @@ __device__ __forceinline__ void group_arrive_wait(unsigned* ctr, unsigned target
 // once every split of the group has its partials -- the score pass over the
 // same split's keys (its K tiles are still in L2) while four warps merge this
 // split's share of the group's output rows, then (fuse_select) the selection
-// of the group's rows by all of the group's CTAs together: each keeps its
-// split's candidate scores in shared memory, adds them to the level-2 and
-// level-3 digit histograms in global memory between group barriers, and
-// writes its survivors at the offset the lower splits' counts give.  Without
-// fuse_select a separate selection kernel follows.
+// of the group's rows by all of the group's CTAs together, each keeping its
+// split's candidate scores in shared memory (two more group barriers; see
+// below).  Without fuse_select a separate selection kernel follows.
 template <int N, int G, bool FP8>
 __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     attn_tc_fused_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -630,6 +630,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   constexpr int W = kThreads / 32;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int s_res[2], s_tmp[32], s_prefix[4], s_need[4], s_base[2];
+  static_assert(W <= 16, "per-warp counters");
   __shared__ int s_wg[4][16], s_we[4][16];
   uint8_t* smem = align1024(smem_raw);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kSlotOff);
@@ -677,12 +678,6 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   unsigned* gsync = p.grp_sync + 8 * grp;
-  if (p.fuse_select && split == 0)  // the group's level-2/3 counters start at zero
-    for (int q = 0; q < G && t0 + q < p.T; ++q) {
-      const long long row = (long long)b * p.T + t0 + q;
-      for (int u = threadIdx.x; u < 2048; u += kThreads) p.hist2[row * 2048 + u] = 0u;
-      for (int u = threadIdx.x; u < 512; u += kThreads) p.hist3[row * 512 + u] = 0u;
-    }
   tc_fence_before();
   group_arrive_wait(gsync, (unsigned)ns);  // the group's partials are out
   tc_fence_after();
@@ -799,11 +794,12 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
 #pragma unroll
         for (int q = 0; q < G; ++q) {
           const int t = t0 + q;
-          if (t < p.T && j <= p.L - p.T + t - p.window) {
+          const bool cand = t < p.T && j <= p.L - p.T + t - p.window;
+          if (cand) {
             p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
             if (p.fuse_select) seg[q * p.split_keys + (int)(j - k_lo)] = acc[q];
-            atomicAdd(&hist_s[q * kHistBins + (__float_as_uint(acc[q]) >> kHistShift)], 1u);
           }
+          hist_inc_warp(hist_s + q * kHistBins, __float_as_uint(acc[q]) >> kHistShift, cand);
         }
       }
       asm volatile("bar.sync 2, 128;" ::: "memory");
@@ -842,78 +838,138 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   __syncthreads();
 
   // ------------------------------------------ selection (whole group)
-  // Three digit levels of the k-th largest score pattern tau, as in
-  // select_topk_kernel: bits [30:20] (the score pass's histogram), [19:9] and
-  // [8:0]; then the ordered compaction of {v > tau} and the first `need` of
-  // {v == tau}.  Every CTA of the group takes every barrier.
+  // The k-th largest score pattern tau, as in select_topk_kernel, in two group
+  // barriers.  (1) Once the level-1 histogram (bits [30:20], built by the
+  // score pass) is complete, every CTA finds the bin b1 holding the k-th
+  // candidate, counts its split's candidates above b1 and writes the ones in
+  // b1 to its slice of the row's list.  (2) Once every split has done so, every
+  // CTA loads the row's whole b1 list (split order) and finds tau and the
+  // number of ties to keep from two more digit levels (bits [19:9], [8:0]) in
+  // shared memory; the list prefix before its own slice gives the survivors of
+  // the lower splits, and it writes its own survivors in position order.
   if (p.fuse_select) {
     const unsigned* segu = reinterpret_cast<const unsigned*>(seg);
+    unsigned* list_s = reinterpret_cast<unsigned*>(smem);                 // the row's b1 list
+    unsigned* h = reinterpret_cast<unsigned*>(smem + SM::kSelWorkOff);    // 2048 counters
+    int* off_s = reinterpret_cast<int*>(smem + SM::kSelWorkOff + 8192);   // [ns + 1] list offsets
     auto row_of = [&](int q) { return (long long)b * p.T + t0 + q; };
     auto nc_of = [&](int q) { return p.L - p.T + t0 + q - p.window + 1; };
     auto active = [&](int q) { return t0 + q < p.T && nc_of(q) > p.topk && p.topk > 0; };
     auto nseg_of = [&](int q) {
       return (int)max(0LL, min((long long)p.split_keys, nc_of(q) - k_lo));
     };
+    auto list_g = [&](int q, int sp) {
+      return p.sel_list + (row_of(q) * ns + sp) * (long long)p.split_keys;
+    };
     group_arrive_wait(gsync + 1, (unsigned)ns);  // level-1 counts complete
 #pragma unroll 1
     for (int q = 0; q < G; ++q)
       if (active(q)) {
         sel_find_bin_global<kThreads, 2048>(p.hist + row_of(q) * kHistBins, p.topk, s_res, s_tmp);
+        const unsigned b1 = (unsigned)s_res[0];
         if (threadIdx.x == 0) {
           s_prefix[q] = s_res[0];
           s_need[q] = s_res[1];
         }
-      }
-    __syncthreads();
-#pragma unroll 1
-    for (int q = 0; q < G; ++q)
-      if (active(q)) {
-        const unsigned pre = (unsigned)s_prefix[q];
-        unsigned* h = p.hist2 + row_of(q) * 2048;
+        // this split's candidates above b1 and in b1, per warp-contiguous part
         const int n = nseg_of(q);
-        for (int u = threadIdx.x; u < n; u += kThreads) {
-          const unsigned v = segu[q * p.split_keys + u];
-          if ((v >> 20) == pre) atomicAdd(h + ((v >> 9) & 2047u), 1u);
+        const int wseg = (n + W - 1) / W;
+        const int w0 = min(n, warp * wseg), w1 = min(n, w0 + wseg);
+        int n_gt = 0, n_in = 0;
+        for (int base = w0; base < w1; base += 32) {
+          const int u = base + lane;
+          const unsigned d = u < w1 ? (segu[q * p.split_keys + u] >> 20) : 0u;
+          n_gt += __popc(__ballot_sync(0xffffffffu, u < w1 && d > b1));
+          n_in += __popc(__ballot_sync(0xffffffffu, u < w1 && d == b1));
         }
+        if (lane == 0) {
+          s_wg[q][warp] = n_gt;
+          s_we[q][warp] = n_in;
+        }
+        __syncthreads();
+        int in_before = 0, gt_tot = 0, in_tot = 0;
+        for (int w = 0; w < W; ++w) {
+          if (w < warp) in_before += s_we[q][w];
+          gt_tot += s_wg[q][w];
+          in_tot += s_we[q][w];
+        }
+        if (threadIdx.x == 0) p.sel_cnt[row_of(q) * ns + split] = make_int2(gt_tot, in_tot);
+        unsigned* lg = list_g(q, split);
+        for (int base = w0; base < w1; base += 32) {
+          const int u = base + lane;
+          const unsigned v = u < w1 ? segu[q * p.split_keys + u] : 0u;
+          const bool in = u < w1 && (v >> 20) == b1;
+          const unsigned m = __ballot_sync(0xffffffffu, in);
+          if (in) lg[in_before + __popc(m & ((1u << lane) - 1u))] = v;
+          in_before += __popc(m);
+        }
+        __syncthreads();  // s_res / s_w* are reused by the next row
       }
-    group_arrive_wait(gsync + 2, (unsigned)ns);  // level-2 counts complete
+    group_arrive_wait(gsync + 2, (unsigned)ns);  // every split's counts and b1 slice are out
 #pragma unroll 1
     for (int q = 0; q < G; ++q)
       if (active(q)) {
-        sel_find_bin_global<kThreads, 2048>(p.hist2 + row_of(q) * 2048, s_need[q], s_res, s_tmp);
-        if (threadIdx.x == 0) {
-          s_prefix[q] = (s_prefix[q] << 11) | s_res[0];
-          s_need[q] = s_res[1];
+        // list offsets of the splits, and this split's survivors-above-b1 base
+        int2 c = make_int2(0, 0);
+        if (threadIdx.x < ns) c = __ldcg(p.sel_cnt + row_of(q) * ns + threadIdx.x);
+        int in_ex, gt_ex;
+        const int m = sel_block_scan<kThreads>(c.y, in_ex, s_tmp);
+        sel_block_scan<kThreads>(c.x, gt_ex, s_tmp);
+        if (threadIdx.x < ns) off_s[threadIdx.x] = in_ex;
+        if (threadIdx.x == ns) off_s[ns] = m;
+        if (threadIdx.x == split) {
+          s_base[0] = gt_ex;  // candidates above b1 in the lower splits
+          s_base[1] = in_ex;  // list index of this split's slice
         }
-      }
-    __syncthreads();
-#pragma unroll 1
-    for (int q = 0; q < G; ++q)
-      if (active(q)) {
-        const unsigned pre = (unsigned)s_prefix[q];
-        unsigned* h = p.hist3 + row_of(q) * 512;
-        const int n = nseg_of(q);
-        for (int u = threadIdx.x; u < n; u += kThreads) {
-          const unsigned v = segu[q * p.split_keys + u];
-          if ((v >> 9) == pre) atomicAdd(h + (v & 511u), 1u);
+        for (int e = threadIdx.x; e < 2048; e += kThreads) h[e] = 0u;
+        __syncthreads();
+        // element e of the row's list: slice sp with off_s[sp] <= e < off_s[sp + 1]
+        const bool in_smem = m <= SM::kSelCap;
+        auto list_at = [&](int e) {
+          int lo = 0, hi = ns - 1;
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (off_s[mid] <= e) lo = mid;
+            else hi = mid - 1;
+          }
+          return __ldcg(list_g(q, lo) + (e - off_s[lo]));
+        };
+        if (in_smem)
+          for (int e = threadIdx.x; e < m; e += kThreads) list_s[e] = list_at(e);
+        __syncthreads();
+        auto val = [&](int e) { return in_smem ? list_s[e] : list_at(e); };
+        // level 2: bits [19:9] of the list (every element is in b1)
+        const int m_pad = (m + kThreads - 1) / kThreads * kThreads;
+        for (int e = threadIdx.x; e < m_pad; e += kThreads) {
+          const unsigned v = e < m ? val(e) : 0u;
+          hist_inc_warp(h, (v >> 9) & 2047u, e < m);
         }
-      }
-    group_arrive_wait(gsync + 3, (unsigned)ns);  // level-3 counts complete
-#pragma unroll 1
-    for (int q = 0; q < G; ++q)
-      if (active(q)) {
-        sel_find_bin_global<kThreads, 512>(p.hist3 + row_of(q) * 512, s_need[q], s_res, s_tmp);
-        if (threadIdx.x == 0) {
-          s_prefix[q] = (s_prefix[q] << 9) | s_res[0];
-          s_need[q] = s_res[1];
+        __syncthreads();
+        sel_find_bin<kThreads>(h, 2048, s_need[q], s_res, s_tmp);
+        const unsigned pre2 = ((unsigned)s_prefix[q] << 11) | (unsigned)s_res[0];
+        const int need2 = s_res[1];
+        for (int e = threadIdx.x; e < 512; e += kThreads) h[e] = 0u;
+        __syncthreads();
+        for (int e = threadIdx.x; e < m_pad; e += kThreads) {
+          const unsigned v = e < m ? val(e) : 0u;
+          hist_inc_warp(h, v & 511u, e < m && (v >> 9) == pre2);
         }
-      }
-    __syncthreads();
-    // counts above / equal to tau of each warp's contiguous part of this split
-#pragma unroll 1
-    for (int q = 0; q < G; ++q)
-      if (active(q)) {
-        const unsigned tau = (unsigned)s_prefix[q];
+        __syncthreads();
+        sel_find_bin<kThreads>(h, 512, need2, s_res, s_tmp);
+        const unsigned tau = (pre2 << 9) | (unsigned)s_res[0];
+        const int need_tau = s_res[1];
+        // survivors of the lower splits' b1 slices: above tau, and ties
+        const int own = s_base[1];
+        int a = 0, tie = 0;
+        for (int e = threadIdx.x; e < own; e += kThreads) {
+          const unsigned v = val(e);
+          a += v > tau;
+          tie += v == tau;
+        }
+        int a_ex, tie_ex;
+        const int a_tot = sel_block_scan<kThreads>(a, a_ex, s_tmp);
+        const int tie_tot = sel_block_scan<kThreads>(tie, tie_ex, s_tmp);
+        // this split's survivors, per warp-contiguous part: v > tau, v == tau
         const int n = nseg_of(q);
         const int wseg = (n + W - 1) / W;
         const int w0 = min(n, warp * wseg), w1 = min(n, w0 + wseg);
@@ -928,50 +984,14 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
           s_wg[q][warp] = n_gt;
           s_we[q][warp] = n_eq;
         }
-      }
-    __syncthreads();
-    if (threadIdx.x < G && active(threadIdx.x)) {
-      int g = 0, e = 0;
-      for (int w = 0; w < W; ++w) {
-        g += s_wg[threadIdx.x][w];
-        e += s_we[threadIdx.x][w];
-      }
-      p.sel_cnt[row_of(threadIdx.x) * ns + split] = make_int2(g, e);
-    }
-    group_arrive_wait(gsync + 4, (unsigned)ns);  // every split's counts are out
-#pragma unroll 1
-    for (int q = 0; q < G; ++q)
-      if (active(q)) {
-        if (warp == 0) {  // survivors of the lower splits
-          int g = 0, e = 0;
-          for (int sp = lane; sp < split; sp += 32) {
-            const int2 c = __ldcg(p.sel_cnt + row_of(q) * ns + sp);
-            g += c.x;
-            e += c.y;
-          }
-#pragma unroll
-          for (int o = 16; o; o >>= 1) {
-            g += __shfl_xor_sync(0xffffffffu, g, o);
-            e += __shfl_xor_sync(0xffffffffu, e, o);
-          }
-          if (lane == 0) {
-            s_base[0] = g;
-            s_base[1] = e;
-          }
-        }
         __syncthreads();
-        const unsigned tau = (unsigned)s_prefix[q];
-        const int need = s_need[q];
-        int gt_before = s_base[0], eq_before = s_base[1];
+        int gt_before = s_base[0] + a_tot, eq_before = tie_tot;
         for (int w = 0; w < warp; ++w) {
           gt_before += s_wg[q][w];
           eq_before += s_we[q][w];
         }
-        const int n = nseg_of(q);
-        const int wseg = (n + W - 1) / W;
-        const int w0 = min(n, warp * wseg), w1 = min(n, w0 + wseg);
         int32_t* out = p.idx + row_of(q) * p.slots;
-        int pos = gt_before + min(eq_before, need);
+        int pos = gt_before + min(eq_before, need_tau);
         int eq_rank = eq_before;
         for (int base = w0; base < w1; base += 32) {
           const int u = base + lane;
@@ -980,7 +1000,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
           const bool eq = u < w1 && v == tau;
           const unsigned eqm = __ballot_sync(0xffffffffu, eq);
           const int my_eq_rank = eq_rank + __popc(eqm & ((1u << lane) - 1u));
-          const bool sel = gt || (eq && my_eq_rank < need);
+          const bool sel = gt || (eq && my_eq_rank < need_tau);
           const unsigned selm = __ballot_sync(0xffffffffu, sel);
           if (sel) {
             const int o = pos + __popc(selm & ((1u << lane) - 1u));
@@ -991,7 +1011,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         }
         if (split == ns - 1 && warp == W - 1 && lane == 0 && pos != p.topk)
           raise_status(kStatusBadIndex);
-        __syncthreads();  // s_base is rewritten for the next row
+        __syncthreads();  // shared state is rewritten for the next row
       }
     if (split == 0)  // window, padding and count; or every position when all are taken
       for (int q = 0; q < G && t0 + q < p.T; ++q) {
@@ -1183,10 +1203,9 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
 #pragma unroll
       for (int q = 0; q < G; ++q) {
         const int t = t0 + q;
-        if (t < p.T && j <= p.L - p.T + t - p.window) {
-          p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
-          atomicAdd(&hist_s[q * kHistBins + (__float_as_uint(acc[q]) >> kHistShift)], 1u);
-        }
+        const bool cand = t < p.T && j <= p.L - p.T + t - p.window;
+        if (cand) p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
+        hist_inc_warp(hist_s + q * kHistBins, __float_as_uint(acc[q]) >> kHistShift, cand);
       }
     }
     softmax_sync<128>();

@@ -44,9 +44,8 @@ struct FullAttnParams {
   // fused tcgen05 pass only: per-group arrival counters (zeroed before the
   // launch), and the selection outputs when the selection is fused too
   unsigned* grp_sync;            // [groups][8]
-  unsigned* hist2;               // [B*T][2048] level-2 counts (fused selection)
-  unsigned* hist3;               // [B*T][512]  level-3 counts
-  int2* sel_cnt;                 // [B*T][splits] (above, equal to) the threshold per split
+  unsigned* sel_list;            // [B*T][splits][split_keys] candidate scores in the level-1 bin
+  int2* sel_cnt;                 // [B*T][splits] candidates above / in the level-1 bin per split
   int32_t* idx;                  // [B*T][slots]
   int32_t* n_sel;                // [B*T]
   int topk, slots, fuse_select;
@@ -493,11 +492,10 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             const long long key = kbase + nt * 8 + 2 * c + j;
-            if (key <= i_q - p.window) {
-              const float v = acc[q][nt][j];
-              srow[key] = v;
-              atomicAdd(&hist_s[q * kHistBins + (__float_as_uint(v) >> kHistShift)], 1u);
-            }
+            const bool cand = key <= i_q - p.window;
+            const float v = acc[q][nt][j];
+            if (cand) srow[key] = v;
+            hist_inc_warp(hist_s + q * kHistBins, __float_as_uint(v) >> kHistShift, cand, 0xFu);
           }
       }
     }

@@ -91,8 +91,8 @@ struct FullPlan {
   int rows;      // query rows per group (N of the tcgen05 tiles, or 32)
   int tile;      // keys per pipeline tile
   int G, groups_per_seq, n_groups, n_splits, split_keys, score_splits, score_keys;
-  size_t off_part_o, off_part_ml, off_lse, off_hist, off_score, off_sync, off_hist2, off_hist3,
-      off_cnt, total;
+  size_t off_part_o, off_part_ml, off_lse, off_hist, off_score, off_sync, off_list, off_cnt,
+      total;
 };
 
 bool check_attn_shape(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt) {
@@ -139,13 +139,11 @@ bool make_full_plan(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt, Full
   off = align_up(off + (size_t)B * T * kHistBins * 4, 256);
   pl->off_score = off;
   off = align_up(off + (size_t)B * T * (size_t)L * 4, 256);
-  pl->off_sync = pl->off_hist2 = pl->off_hist3 = pl->off_cnt = off;
+  pl->off_sync = pl->off_list = pl->off_cnt = off;
   if (pl->fused) {
     off = align_up(off + (size_t)pl->n_groups * 8 * 4, 256);
-    pl->off_hist2 = off;
-    off = align_up(off + (size_t)B * T * 2048 * 4, 256);
-    pl->off_hist3 = off;
-    off = align_up(off + (size_t)B * T * 512 * 4, 256);
+    pl->off_list = off;
+    off = align_up(off + (size_t)B * T * pl->n_splits * pl->split_keys * 4, 256);
     pl->off_cnt = off;
     off = align_up(off + (size_t)B * T * pl->n_splits * 8, 256);
   }
@@ -267,7 +265,8 @@ hs2_status run_fused_tc(const CUtensorMap& km, const CUtensorMap& vm, FullAttnPa
   static_assert(SM::kBytes <= 232448, "shared memory per CTA");
   // the selection is fused when a split's candidate scores of the group's
   // rows fit the P^T buffers (shared memory free after the partial pass)
-  fp.fuse_select = (long long)fp.G * fp.split_keys * 4 <= SM::kNP * SM::kPBytes;
+  fp.fuse_select = (long long)fp.G * fp.split_keys * 4 <= SM::kNP * SM::kPBytes &&
+                   pl.n_splits <= 256;
   auto kf = fp.G == 1 ? attn_tc_fused_kernel<32, 1, FP8>
                       : (fp.G == 2 ? attn_tc_fused_kernel<32, 2, FP8>
                                    : attn_tc_fused_kernel<32, 4, FP8>);
@@ -405,8 +404,7 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
   sp.cs = 1;
 
   fp.grp_sync = reinterpret_cast<unsigned*>(ws + pl.off_sync);
-  fp.hist2 = reinterpret_cast<unsigned*>(ws + pl.off_hist2);
-  fp.hist3 = reinterpret_cast<unsigned*>(ws + pl.off_hist3);
+  fp.sel_list = reinterpret_cast<unsigned*>(ws + pl.off_list);
   fp.sel_cnt = reinterpret_cast<int2*>(ws + pl.off_cnt);
   fp.idx = idx;
   fp.n_sel = n_sel;

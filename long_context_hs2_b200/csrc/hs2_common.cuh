@@ -157,6 +157,18 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two) {
   return pack_bf16(f.x, f.y);
 }
 
+// Warp-aggregated histogram increment in shared memory: every lane with
+// `active` adds 1 to h[bin]; lanes that share a bin are combined into one
+// atomic by the lowest of them.  Every lane of `lanes` must call it.
+__device__ __forceinline__ void hist_inc_warp(unsigned* h, unsigned bin, bool active,
+                                              unsigned lanes = 0xffffffffu) {
+  const unsigned act = __ballot_sync(lanes, active);
+  if (active) {
+    const unsigned peers = __match_any_sync(act, bin);
+    if ((threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1)) atomicAdd(h + bin, (unsigned)__popc(peers));
+  }
+}
+
 // ----------------------------------------------- 128B-swizzled bf16 tiles --
 // A [N][D] bf16 tile is stored as D/64 column halves; half h holds columns
 // 64h .. 64h+63 of every row as N rows of 128 bytes, and the 16-byte chunk c

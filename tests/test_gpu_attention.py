@@ -143,3 +143,31 @@ def test_chunk_bf16_h32_wide_groups():
     wl = WORKLOADS["decode_bf16_32k"].resized(B=2, T=70, L=9000, n_needles=20, n_sparse=1)
     rows = np.unique(np.r_[0, 69, 70, 139, np.random.default_rng(2).integers(0, 140, 24)])
     _check_block(wl, rows=rows)
+
+
+def test_fused_short_context_and_zero_topk():
+    # head_dim 128 takes the fused kernel: contexts whose candidates all fit
+    # the budget, and a zero budget (the window alone)
+    wl = WORKLOADS["decode_bf16_32k"].resized(B=2, T=3, L=100, n_needles=0, topk=16, window=128)
+    _check_block(wl, needles=False)
+    wl = WORKLOADS["decode_bf16_32k"].resized(B=2, T=2, L=700, n_needles=0, topk=0, window=32)
+    _check_block(wl, needles=False)
+
+
+def test_all_scores_tied_large_context():
+    # identical keys: every candidate score is the same pattern, so the
+    # selection is decided by position alone (lowest positions first), and the
+    # level-1 bin holds every candidate (more than the fused selection keeps
+    # in shared memory)
+    wl = WORKLOADS["decode_bf16_32k"].resized(B=1, L=65536, n_needles=0, n_sparse=1)
+    inp = make_attention_inputs(wl, needles=False)
+    inp.k[:] = inp.k[:, :1, :]
+    di = tl.DeviceInputs(inp)
+    g = tl.run_full(di)
+    orc = tl.oracle_full(inp, rows=np.arange(1))
+    i = wl.L - 1
+    want = np.r_[np.arange(wl.topk), np.arange(i - wl.window + 1, i + 1)]
+    assert np.array_equal(orc["idx"][0, : orc["n_sel"][0]], want)
+    assert int(g["n_sel"][0]) == want.size
+    assert np.array_equal(g["idx"][0, : want.size], want)
+    assert tl.max_abs(g["o"][:1], orc["o"]) <= tl.TOL_BF16
