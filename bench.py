@@ -129,6 +129,30 @@ def dist_setup():
     return world, rank, local
 
 
+# Multi-GPU runs are replicas: the decode path shards by sequence with no
+# exchange, so rank r runs its own sequences (the workload with its seed moved
+# by r) and the only collectives are barriers and the max-over-ranks timing.
+def rank_workload(rank: int):
+    base = WORKLOADS[WORKLOAD]
+    return base.resized(seed=base.seed + 1000 * rank)
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest of every rank's `value` (a no-op for one rank)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms * 1e-3)
+
+
 # ------------------------------------------------------------- oracle arm --
 def oracle_rows_per_s(inp, rows, n_sparse):
     """Oracle time for the block on `rows` query rows (full + select + sparse layers)."""
@@ -274,8 +298,7 @@ def run_hs2(args, world, rank, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     hs2.load_library()
-    base = WORKLOADS[WORKLOAD]
-    wl = base.resized(seed=base.seed + 1000 * rank)       # each rank: its own sequences
+    wl = rank_workload(rank)       # each rank: its own sequences
     inp = make_attention_inputs(wl)
     B, T, L, H, D = wl.B, wl.T, wl.L, wl.H, wl.D
     slots = wl.topk + wl.window
@@ -418,12 +441,7 @@ def run_hs2(args, world, rank, local):
     e2e_ms = [a.elapsed_time(c) for a, c in e2e_ev]
 
     def agg(xs):
-        m = float(np.mean(xs))
-        if world > 1:
-            t = torch.tensor([m], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            m = float(t.item())
-        return m
+        return max_over_ranks(float(np.mean(xs)), world, "cuda")
 
     ms = agg(step_ms)
     full = agg(full_ms)
@@ -451,10 +469,9 @@ def run_hs2(args, world, rank, local):
         dist.destroy_process_group()
     if rank != 0:
         return
-    tokens = B * T * world
     line = {
         "metric": "hybrid-block decode tokens/s",
-        "value": tokens / (ms * 1e-3),
+        "value": job_throughput(B * T, world, ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -469,7 +486,8 @@ def run_hs2(args, world, rank, local):
                    "kv": "bf16", "topk": wl.topk, "window": wl.window,
                    "sparse_layers": wl.n_sparse, "parallelism": "replicas (dp%d)" % world,
                    "l2": "flushed before each step (512 MB write, then read back)"},
-        "e2e": {"value": tokens / (e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_throughput(B * T, world, e2e), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         # per step: the fused full-attention kernel (partials, score and
         # selection in one launch for this shape) and one per sparse layer
