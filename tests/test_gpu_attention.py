@@ -22,8 +22,8 @@ def _positions(wl, rows):
     return [wl.L - wl.T + (r % wl.T) for r in rows]
 
 
-def _check_block(wl, rows=None, sparse_layers=None, needles=True):
-    inp = make_attention_inputs(wl, needles=needles)
+def _check_block(wl, rows=None, sparse_layers=None, needles=True, inp=None):
+    inp = make_attention_inputs(wl, needles=needles) if inp is None else inp
     di = tl.DeviceInputs(inp)
     g = tl.run_full(di)
     rows = np.arange(wl.B * wl.T) if rows is None else np.asarray(rows)
@@ -171,3 +171,14 @@ def test_all_scores_tied_large_context():
     assert int(g["n_sel"][0]) == want.size
     assert np.array_equal(g["idx"][0, : want.size], want)
     assert tl.max_abs(g["o"][:1], orc["o"]) <= tl.TOL_BF16
+
+
+def test_chunk_fp8_1m_sampled_rows():
+    # the full 4096-query chunk over a 1M-token E4M3 cache, in the launch
+    # configuration of that shape; the oracle checks sampled query rows (first,
+    # middle, last, and rows that own planted needles) one by one
+    wl = WORKLOADS["chunk_fp8_1m"].resized(n_sparse=1)
+    inp = make_attention_inputs(wl)
+    needle_rows = sorted({int(t) for _, _, t in inp.needles})[:: max(1, len(inp.needles) // 3)][:3]
+    rows = np.unique(np.r_[0, 1, wl.T // 2, wl.T - 1, needle_rows])
+    _check_block(wl, rows=rows, inp=inp)
