@@ -181,7 +181,7 @@ HS2_API hs2_status hs2_sparse_attn(const void* Q, const hs2_kv_cache* kv, int B,
  *     first call before any stream capture on the device.
  *   - A request whose workspace (hs2_full_attn_select_workspace) exceeds
  *     HS2_NOALLOC_SCRATCH_BYTES returns HS2_ERR_WORKSPACE and enqueues nothing.
- *     For example, 8 sequences of 32K positions need about 3.6 MB.
+ *     For example, 8 sequences of 32K positions need about 4.6 MB.
  *   - All calls on a device share the one array, and it keeps whatever the
  *     last call left there; the kernels clear the parts that must start at
  *     zero themselves.  Calls whose work overlaps on the GPU (different
