@@ -641,6 +641,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   uint64_t* k2_full = s2_empty + 2;    // [2], E4M3 only
   uint64_t* k2_free = k2_full + 2;     // [2]
 
+  pdl_launch_dependents();  // a following sparse layer may place its CTAs on idle SMs
   tc_partial_setup<N, FP8>(smem);
   if (threadIdx.x == 0) {
     for (int s = 0; s < S2; ++s) {

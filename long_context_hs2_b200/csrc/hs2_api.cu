@@ -156,13 +156,13 @@ bool make_full_plan(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt, Full
 // fails) when coop.
 template <typename... KArgs, typename... Args>
 hs2_status launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                     int cluster, bool coop, Args&&... args) {
+                     int cluster, bool coop, bool pdl, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   int na = 0;
   if (cluster > 1) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
@@ -174,6 +174,11 @@ hs2_status launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
   if (coop) {
     attr[na].id = cudaLaunchAttributeCooperative;
     attr[na].val.cooperative = 1;
+    ++na;
+  }
+  if (pdl) {  // may start before the previous kernel ends; the kernel waits on it itself
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
   }
   cfg.attrs = attr;
@@ -188,7 +193,8 @@ hs2_status launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
 template <typename... KArgs, typename... Args>
 hs2_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                   int cluster, Args&&... args) {
-  return launch_ex(kernel, grid, block, smem, s, cluster, false, std::forward<Args>(args)...);
+  return launch_ex(kernel, grid, block, smem, s, cluster, false, false,
+                   std::forward<Args>(args)...);
 }
 
 template <typename K>
@@ -277,7 +283,7 @@ hs2_status run_fused_tc(const CUtensorMap& km, const CUtensorMap& vm, FullAttnPa
   }
   if (stage_mark(s, true) != cudaSuccess) return HS2_ERR_CUDA;
   const hs2_status st = launch_ex(kf, dim3(pl.n_groups * pl.n_splits), dim3(tc_partial_threads(FP8)),
-                                  SM::kBytes, s, 1, pl.n_splits > 1, km, vm, fp);
+                                  SM::kBytes, s, 1, pl.n_splits > 1, false, km, vm, fp);
   if (st != HS2_OK) return st;
   if (stage_mark(s, false) != cudaSuccess) return HS2_ERR_CUDA;
   return fp.fuse_select ? HS2_OK : run_select(fp, sp, s);
@@ -288,8 +294,8 @@ hs2_status run_sparse(const SparseParams& p, cudaStream_t s) {
   using SM = SparseSmem<MT, D, FP8>;
   auto k = sparse_attn_kernel<MT, D, FP8>;
   if (!set_smem(k, SM::kBytes)) return HS2_ERR_CUDA;
-  return launch(k, dim3((unsigned)((long long)p.B * p.T * p.cs)), dim3(128), SM::kBytes, s, p.cs,
-                p);
+  return launch_ex(k, dim3((unsigned)((long long)p.B * p.T * p.cs)), dim3(128), SM::kBytes, s,
+                   p.cs, false, true, p);
 }
 
 }  // namespace

@@ -157,6 +157,15 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two) {
   return pack_bf16(f.x, f.y);
 }
 
+// Programmatic dependent launch: let the next kernel of the stream (launched
+// with programmatic stream serialization) start its CTAs now, and wait until
+// every kernel this one depends on has completed and its memory is visible.
+// Both are no-ops for kernels launched without that attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Warp-aggregated histogram increment in shared memory: every lane with
 // `active` adds 1 to h[bin]; lanes that share a bin are combined into one
 // atomic by the lowest of them.  Every lane of `lanes` must call it.

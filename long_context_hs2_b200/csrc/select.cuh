@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
   __shared__ int wsel[kSelThreads / 32], weq[kSelThreads / 32];
   extern __shared__ unsigned seg_s[];
 
+  pdl_launch_dependents();  // a following sparse layer may place its CTAs on idle SMs
   const int cs = p.cs;
   const uint32_t rank = cs > 1 ? sel_cluster_rank() : 0u;
   const long long row = blockIdx.x / cs;

@@ -118,6 +118,8 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   float* cl_o = reinterpret_cast<float*>(smem + SM::kClOff + SM::kRowsQ * 8);
   int* pos_all = reinterpret_cast<int*>(smem + SM::kPosOff);  // [my_tiles][64]
 
+  pdl_launch_dependents();
+  pdl_wait();  // indices, counts and queries come from earlier kernels
   const int cs = p.cs;
   const uint32_t rank = cs > 1 ? cluster_ctarank() : 0u;
   const long long qrow = blockIdx.x / cs;  // b*T + t
