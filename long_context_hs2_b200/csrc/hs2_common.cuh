@@ -166,16 +166,13 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Warp-aggregated histogram increment in shared memory: every lane with
-// `active` adds 1 to h[bin]; lanes that share a bin are combined into one
-// atomic by the lowest of them.  Every lane of `lanes` must call it.
+// Histogram increment in shared memory by every lane with `active` (plain
+// atomics: on B200 they beat combining equal bins with __match_any_sync).
+// Every lane of `lanes` calls it.
 __device__ __forceinline__ void hist_inc_warp(unsigned* h, unsigned bin, bool active,
                                               unsigned lanes = 0xffffffffu) {
-  const unsigned act = __ballot_sync(lanes, active);
-  if (active) {
-    const unsigned peers = __match_any_sync(act, bin);
-    if ((threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1)) atomicAdd(h + bin, (unsigned)__popc(peers));
-  }
+  (void)lanes;
+  if (active) atomicAdd(h + bin, 1u);
 }
 
 // ----------------------------------------------- 128B-swizzled bf16 tiles --
