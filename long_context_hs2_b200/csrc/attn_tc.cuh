@@ -249,14 +249,25 @@ __device__ __forceinline__ void tc_partial_setup(uint8_t* smem) {
   }
 }
 
+// Tiles whose logits stay in tensor memory in a retaining partial pass (32
+// columns each beside the 32 of O^T: all 512 columns).
+constexpr int kTcRetainTiles = 15;
+
 // The partial pass of one (group, split) work item: every role's work, with
-// the barriers of tc_partial_setup initialised and 4N TMEM columns at `tmem`.
+// the barriers of tc_partial_setup initialised and the TMEM columns at `tmem`
+// (4N; 512 when RETAIN).  TMEM layout: S^T double buffer at columns 0 and N,
+// O^T at 2N, per-key row sums at 3N; with RETAIN (N = 32, at most
+// kTcRetainTiles tiles) O^T at 0 and the S^T of tile n kept at N + n*N for a
+// later score pass, the row sums in registers.
 // Returns in every thread once its role is done (no trailing barrier).
-template <int N, int G, bool FP8>
+template <int N, int G, bool FP8, bool RETAIN = false>
 __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const CUtensorMap& vmap,
                                                 const FullAttnParams& p, uint8_t* smem,
                                                 uint32_t tmem) {
+  static_assert(!RETAIN || N == 32, "retained logits: 32 rows per group");
   using SM = TcSmem<N, FP8>;
+  constexpr uint32_t kOCol = RETAIN ? 0 : 2 * N;
+  auto s_col = [](int n) -> uint32_t { return RETAIN ? N + n * N : (n & 1) * N; };
   constexpr int S = SM::kStages;
   constexpr int NP = SM::kNP;
   constexpr int kH = N / G;     // heads per query
@@ -335,7 +346,7 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
         if (!mbar_wait(&p_full[m % NP], (m / NP) & 1)) return false;
         if (FP8 && !mbar_wait(v16_full, m & 1)) return false;
         tc_fence_after();
-        tc_issue_pv<N, FP8>(tmem + 2 * N,
+        tc_issue_pv<N, FP8>(tmem + kOCol,
                             FP8 ? v16_addr : smem_u32(smem + (m % S) * SM::kStageBytes + kTileIn),
                             p_addr + (m % NP) * SM::kPBytes, m > 0);
         tc_commit(&pv_done[m % NP]);
@@ -346,9 +357,9 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
       for (int n = 0; n < n_tiles && ok; ++n) {
         const int s = n % S, bb = n & 1;
         if (!mbar_wait(FP8 ? k16_full : &kv_full[s], FP8 ? (n & 1) : (n / S) & 1)) break;
-        if (n >= 2 && !mbar_wait(&s_empty[bb], ((n - 2) >> 1) & 1)) break;
+        if (!RETAIN && n >= 2 && !mbar_wait(&s_empty[bb], ((n - 2) >> 1) & 1)) break;
         tc_fence_after();
-        tc_issue_qk<N, FP8>(tmem + bb * N, FP8 ? k16_addr : smem_u32(smem + s * SM::kStageBytes),
+        tc_issue_qk<N, FP8>(tmem + s_col(n), FP8 ? k16_addr : smem_u32(smem + s * SM::kStageBytes),
                             q_addr);
         tc_commit(&s_full[bb]);
         if (FP8) tc_commit(k16_free);
@@ -400,7 +411,10 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
 #pragma unroll
     for (int m = 0; m < 8; ++m) xoff[m] = ((((keyrow & 63) >> 3) ^ m) << 4) + (keyrow & 7) * 2;
     bool failed = false;
-    {  // TMEM is undefined at allocation: clear this thread's row sums
+    float lreg[RETAIN ? NC : 1];  // RETAIN: this key's row sums in registers
+#pragma unroll
+    for (int i = 0; i < (RETAIN ? NC : 1); ++i) lreg[i] = 0.f;
+    if (!RETAIN) {  // TMEM is undefined at allocation: clear this thread's row sums
       float z[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) z[i] = 0.f;
@@ -427,7 +441,7 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
       long long limit[G];
 #pragma unroll
       for (int q = 0; q < G; ++q) limit[q] = min(k_hi - 1, p.L - p.T + t0 + q);
-      const uint32_t s_addr = tmem + lane_base + bb * N + c0;
+      const uint32_t s_addr = tmem + lane_base + s_col(n) + c0;
       // sweep 1: does any logit exceed its row's reference by more than 2^8?
       bool need = false;
 #pragma unroll
@@ -478,17 +492,22 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
 #pragma unroll
         for (int c = 0; c < NC; c += 16) {
           float v[16];
-          tmem_ld16(tmem + lane_base + 3 * N + c0 + c, v);
-          tmem_ld_wait();
+          if (RETAIN) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] *= corr[c0 + c + i];
-          tmem_st16(tmem + lane_base + 3 * N + c0 + c, v);
-          if (n >= 1) {
-            tmem_ld16(tmem + lane_base + 2 * N + c0 + c, v);
+            for (int i = 0; i < 16; ++i) lreg[(c + i) % (RETAIN ? NC : 1)] *= corr[c0 + c + i];
+          } else {
+            tmem_ld16(tmem + lane_base + 3 * N + c0 + c, v);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] *= corr[c0 + c + i];
-            tmem_st16(tmem + lane_base + 2 * N + c0 + c, v);
+            tmem_st16(tmem + lane_base + 3 * N + c0 + c, v);
+          }
+          if (n >= 1) {
+            tmem_ld16(tmem + lane_base + kOCol + c0 + c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] *= corr[c0 + c + i];
+            tmem_st16(tmem + lane_base + kOCol + c0 + c, v);
           }
         }
       }
@@ -499,7 +518,12 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
       for (int c = 0; c < NC; c += 16) {
         float x[16], lv[16];
         tmem_ld16(s_addr + c, x);
-        tmem_ld16(tmem + lane_base + 3 * N + c0 + c, lv);
+        if (RETAIN) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) lv[i] = lreg[(c + i) % (RETAIN ? NC : 1)];
+        } else {
+          tmem_ld16(tmem + lane_base + 3 * N + c0 + c, lv);
+        }
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -515,7 +539,12 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
             *reinterpret_cast<__nv_bfloat16*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
                 __float2bfloat16_rn(pr);
         }
-        tmem_st16(tmem + lane_base + 3 * N + c0 + c, lv);
+        if (RETAIN) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) lreg[(c + i) % (RETAIN ? NC : 1)] = lv[i];
+        } else {
+          tmem_st16(tmem + lane_base + 3 * N + c0 + c, lv);
+        }
       }
       tmem_st_wait();
       fence_proxy_async_smem();
@@ -534,8 +563,13 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
 #pragma unroll
       for (int c = 0; c < NC; c += 16) {
         float v[16];
-        tmem_ld16(tmem + lane_base + 3 * N + c0 + c, v);
-        tmem_ld_wait();
+        if (RETAIN) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = lreg[(c + i) % (RETAIN ? NC : 1)];
+        } else {
+          tmem_ld16(tmem + lane_base + 3 * N + c0 + c, v);
+          tmem_ld_wait();
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float s = warp_sum(v[i]);
@@ -545,7 +579,7 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
 #pragma unroll
       for (int c = 0; c < NC; c += 16) {
         float v[16];
-        tmem_ld16(tmem + lane_base + 2 * N + c0 + c, v);
+        tmem_ld16(tmem + lane_base + kOCol + c0 + c, v);
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 16; ++i) p.part_o[(part * N + c0 + c + i) * 128 + keyrow] = v[i];
@@ -618,10 +652,11 @@ __device__ __forceinline__ void group_arrive_wait(unsigned* ctr, unsigned target
 // of the group's rows by all of the group's CTAs together, each keeping its
 // split's candidate scores in shared memory (two more group barriers; see
 // below).  Without fuse_select a separate selection kernel follows.
-template <int N, int G, bool FP8>
+template <int N, int G, bool FP8, bool RETAIN>
 __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     attn_tc_fused_kernel(const __grid_constant__ CUtensorMap kmap,
                          const __grid_constant__ CUtensorMap vmap, const FullAttnParams p) {
+  constexpr uint32_t kTmemCols = RETAIN ? 512 : 4 * N;
   using SM = TcSmem<N, FP8>;
   static_assert(SM::kFusable, "score pass does not fit the tile ring");
   constexpr int kThreads = tc_partial_threads(FP8);
@@ -657,7 +692,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     fence_mbar_init();
   }
   if (threadIdx.x / 32 == 1) {
-    tmem_alloc(tmem_slot, 4 * N);
+    tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -666,7 +701,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   const uint32_t tmem = *tmem_slot;
 
   // ------------------------------------------------------------ partials
-  tc_partial_body<N, G, FP8>(kmap, vmap, p, smem, tmem);
+  tc_partial_body<N, G, FP8, RETAIN>(kmap, vmap, p, smem, tmem);
 
   const int ns = p.n_splits;
   const int split = blockIdx.x % ns;
@@ -692,8 +727,9 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   uint8_t* k16 = smem + SM::kK16Off;  // E4M3: two f16 K tiles
   // fuse_select: this split's candidate scores of row q at seg[q * split_keys + (j - k_lo)]
   float* seg = reinterpret_cast<float*>(smem + SM::kPOff);
+  // RETAIN: the logits of every tile are still in TMEM: no loads, no MMA
   if (warp == 0) {
-    if (lane == 0) {
+    if (lane == 0 && !RETAIN) {
       const uint64_t pol = policy_evict_first();
       for (int n = 0; n < n2; ++n) {
         const int s = n % S2;
@@ -706,7 +742,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && !RETAIN) {
       const uint32_t q_addr = smem_u32(smem + SM::kQOff);
       for (int n = 0; n < n2; ++n) {
         const int s = n % S2, bb = n & 1;
@@ -728,7 +764,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   } else if (FP8 && warp >= 2 + kTcSoftmax / 32) {
     // E4M3 -> f16: converter warp 10 + i takes key rows 32i .. 32i+31 of a tile
     const int i = warp - (2 + kTcSoftmax / 32);
-    if (i < 4)
+    if (i < 4 && !RETAIN)
       for (int n = 0; n < n2; ++n) {
         const int s = n % S2, bb = n & 1;
         if (!mbar_wait(&kv2_full[s], (n / S2) & 1)) break;
@@ -775,15 +811,16 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         const long long j = k_lo + (long long)n * kTcKeys + keyrow;
         float sl = p.scale_log2;
         if (FP8) sl *= j < k2_hi ? p.k_scale[(long long)b * p.L + j] : 0.f;
-        if (!mbar_wait(&s2_full[bb], (n >> 1) & 1)) break;
+        if (!RETAIN && !mbar_wait(&s2_full[bb], (n >> 1) & 1)) break;
         tc_fence_after();
+        const uint32_t s_col = RETAIN ? N + n * N : bb * N;
         float acc[G];
 #pragma unroll
         for (int q = 0; q < G; ++q) acc[q] = 0.f;
 #pragma unroll
         for (int c = 0; c < N / 32; ++c) {
           float x[32];
-          tmem_ld32(tmem + lane_base + bb * N + 32 * c, x);
+          tmem_ld32(tmem + lane_base + s_col + 32 * c, x);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i)
@@ -791,7 +828,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s2_empty[bb]);
+        if (!RETAIN && lane == 0) mbar_arrive(&s2_empty[bb]);
 #pragma unroll
         for (int q = 0; q < G; ++q) {
           const int t = t0 + q;
@@ -1034,7 +1071,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 4 * N);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 

@@ -273,9 +273,15 @@ hs2_status run_fused_tc(const CUtensorMap& km, const CUtensorMap& vm, FullAttnPa
   // rows fit the P^T buffers (shared memory free after the partial pass)
   fp.fuse_select = (long long)fp.G * fp.split_keys * 4 <= SM::kNP * SM::kPBytes &&
                    pl.n_splits <= 256;
-  auto kf = fp.G == 1 ? attn_tc_fused_kernel<32, 1, FP8>
-                      : (fp.G == 2 ? attn_tc_fused_kernel<32, 2, FP8>
-                                   : attn_tc_fused_kernel<32, 4, FP8>);
+  // the logits of every tile stay in TMEM for the score pass when a split has
+  // at most kTcRetainTiles tiles
+  const bool retain = (fp.split_keys + kTcKeys - 1) / kTcKeys <= kTcRetainTiles;
+  auto kf = retain ? (fp.G == 1 ? attn_tc_fused_kernel<32, 1, FP8, true>
+                                : (fp.G == 2 ? attn_tc_fused_kernel<32, 2, FP8, true>
+                                             : attn_tc_fused_kernel<32, 4, FP8, true>))
+                   : (fp.G == 1 ? attn_tc_fused_kernel<32, 1, FP8, false>
+                                : (fp.G == 2 ? attn_tc_fused_kernel<32, 2, FP8, false>
+                                             : attn_tc_fused_kernel<32, 4, FP8, false>));
   if (!set_smem(kf, SM::kBytes)) return HS2_ERR_CUDA;
   if (cudaMemsetAsync(fp.grp_sync, 0, (size_t)pl.n_groups * 8 * 4, s) != cudaSuccess) {
     cudaGetLastError();

@@ -182,3 +182,9 @@ def test_chunk_fp8_1m_sampled_rows():
     needle_rows = sorted({int(t) for _, _, t in inp.needles})[:: max(1, len(inp.needles) // 3)][:3]
     rows = np.unique(np.r_[0, 1, wl.T // 2, wl.T - 1, needle_rows])
     _check_block(wl, rows=rows, inp=inp)
+
+
+def test_decode_bf16_64k_many_tiles_per_split():
+    # 29 key tiles per split: more than tensor memory keeps, so the fused
+    # kernel's score pass recomputes the logits from K (bf16 cache)
+    _check_block(WORKLOADS["decode_bf16_32k"].resized(L=65536, n_needles=32), sparse_layers=[0])
