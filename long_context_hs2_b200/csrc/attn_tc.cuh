@@ -65,7 +65,9 @@ struct TcSmem {
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBar2Off = kSlotOff + 16;         // fused kernel: score-pass barriers
   static constexpr int kNumBars2 = 16;
-  static constexpr int kBytes = kBar2Off + kNumBars2 * 8 + 1024;
+  static constexpr int kMhistOff = kBar2Off + kNumBars2 * 8;  // retained tiles' references
+  static constexpr int kMhistBytes = N == 32 ? 15 * N * 4 : 0;
+  static constexpr int kBytes = kMhistOff + kMhistBytes + 1024;
   // fused kernel: the score pass reuses the partial pass's tile ring for its
   // K ring, the group's (m, l) partials and the histograms; the fused
   // selection then uses it for the row's candidate scores and its counters
@@ -512,11 +514,14 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
         }
       }
       // sweep 2: p = 2^(x - m_ref), row sums, P^T (bf16, or f16 times the
-      // value scale for an E4M3 cache) for the PV product
+      // value scale for an E4M3 cache) for the PV product; RETAIN: p replaces
+      // the logits in the tile's TMEM block, with the tile's reference kept
       uint8_t* pt = p_base + (n % NP) * SM::kPBytes;
+      if (RETAIN && st < N)
+        reinterpret_cast<float*>(smem + SM::kMhistOff)[n * N + st] = m_ref[st];
 #pragma unroll
       for (int c = 0; c < NC; c += 16) {
-        float x[16], lv[16];
+        float x[16], lv[16], pk[16];
         tmem_ld16(s_addr + c, x);
         if (RETAIN) {
 #pragma unroll
@@ -531,6 +536,7 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
           const bool ok = full_tile || j <= limit[(c + i) / kH + c0 / kH];
           const float mr = m_ref[col];
           const float pr = (ok && mr != kNegInf) ? fast_exp2(x[i] * sl - mr) : 0.f;
+          pk[i] = pr;
           lv[i] += pr;
           if (FP8)
             *reinterpret_cast<__half*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
@@ -542,6 +548,7 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
         if (RETAIN) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) lreg[(c + i) % (RETAIN ? NC : 1)] = lv[i];
+          tmem_st16(s_addr + c, pk);
         } else {
           tmem_st16(tmem + lane_base + 3 * N + c0 + c, lv);
         }
@@ -798,6 +805,16 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       lse2_s[r] = M + log2f(lt);
     }
     softmax_sync<kTcSoftmax>();
+    // RETAIN: TMEM holds p = 2^(x - m_ref(tile)); f[tile][r] = 2^(m_ref(tile) - lse)
+    // turns it into the softmax probability
+    float* fct = reinterpret_cast<float*>(smem + SM::kMhistOff);
+    if (RETAIN) {
+      for (int u = st; u < n2 * N; u += kTcSoftmax) {
+        const float mr = fct[u];
+        fct[u] = mr == kNegInf ? 0.f : fast_exp2(mr - lse2_s[u % N]);
+      }
+      softmax_sync<kTcSoftmax>();
+    }
     if (warp < 6) {
       // ---- score warps 2-5: one key (TMEM lane) each per tile
       const int sc = threadIdx.x - 64;
@@ -810,7 +827,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         const int bb = n & 1;
         const long long j = k_lo + (long long)n * kTcKeys + keyrow;
         float sl = p.scale_log2;
-        if (FP8) sl *= j < k2_hi ? p.k_scale[(long long)b * p.L + j] : 0.f;
+        if (FP8 && !RETAIN) sl *= j < k2_hi ? p.k_scale[(long long)b * p.L + j] : 0.f;
         if (!RETAIN && !mbar_wait(&s2_full[bb], (n >> 1) & 1)) break;
         tc_fence_after();
         const uint32_t s_col = RETAIN ? N + n * N : bb * N;
@@ -822,9 +839,14 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
           float x[32];
           tmem_ld32(tmem + lane_base + s_col + 32 * c, x);
           tmem_ld_wait();
+          if (RETAIN) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            acc[(32 * c + i) / kH] += fast_exp2(x[i] * sl - lse2_s[32 * c + i]);
+            for (int i = 0; i < 32; ++i) acc[(32 * c + i) / kH] += x[i] * fct[n * N + 32 * c + i];
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              acc[(32 * c + i) / kH] += fast_exp2(x[i] * sl - lse2_s[32 * c + i]);
+          }
         }
         tc_fence_before();
         __syncwarp();
