@@ -61,7 +61,7 @@ struct TcSmem {
   static constexpr int kCorrOff = kMrefOff + N * 4;      // float [N]
   static constexpr int kTmaxOff = kCorrOff + N * 4;      // float [4][N] (also the row sums)
   static constexpr int kBarOff = kTmaxOff + 4 * N * 4;
-  static constexpr int kNumBars = 2 * kStages + 9 + 2 * kNP;
+  static constexpr int kNumBars = 3 * kStages + 9 + 2 * kNP;  // + V arrival per stage
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBar2Off = kSlotOff + 16;         // fused kernel: score-pass barriers
   static constexpr int kNumBars2 = 16;
@@ -247,6 +247,7 @@ __device__ __forceinline__ void tc_partial_setup(uint8_t* smem) {
     mbar_init(q_ready + 2, 1);                // k16_free
     mbar_init(q_ready + 3, kTcConvert / 32);  // v16_full
     mbar_init(q_ready + 4, 1);                // v16_free
+    for (int s = 0; s < S; ++s) mbar_init(q_ready + 5 + s, 1);  // v_full (bf16: V of stage s)
     fence_mbar_init();
   }
 }
@@ -289,6 +290,7 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
   uint64_t* k16_free = k16_full + 1;
   uint64_t* v16_full = k16_free + 1;
   uint64_t* v16_free = v16_full + 1;
+  uint64_t* v_full = v16_free + 1;   // [S] bf16: V of a stage (kv_full then means K)
 
   const int split = blockIdx.x % p.n_splits;
   const int grp = blockIdx.x / p.n_splits;
@@ -325,16 +327,18 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
         const int s = n % S;
         if (n >= S && !mbar_wait(&kv_empty[s], ((n / S) - 1) & 1)) break;
         uint8_t* st = smem + s * SM::kStageBytes;
-        mbar_arrive_expect_tx(&kv_full[s], SM::kStageBytes);
         const int row = (int)((long long)b * p.L + k_lo + (long long)n * kTcKeys);
-        if (FP8) {  // 128-byte E4M3 rows: one box per tensor
+        if (FP8) {  // 128-byte E4M3 rows: one box per tensor, both on kv_full
+          mbar_arrive_expect_tx(&kv_full[s], SM::kStageBytes);
           tma_load_2d(st, &kmap, &kv_full[s], 0, row, pol_k);
           tma_load_2d(st + kTileIn, &vmap, &kv_full[s], 0, row, pol_v);
-        } else {
+        } else {  // K on kv_full, V on v_full: QK(n) need not wait for V(n)
+          mbar_arrive_expect_tx(&kv_full[s], kTileIn);
           tma_load_2d(st, &kmap, &kv_full[s], 0, row, pol_k);
           tma_load_2d(st + 16384, &kmap, &kv_full[s], 64, row, pol_k);
-          tma_load_2d(st + kTileIn, &vmap, &kv_full[s], 0, row, pol_v);
-          tma_load_2d(st + kTileIn + 16384, &vmap, &kv_full[s], 64, row, pol_v);
+          mbar_arrive_expect_tx(&v_full[s], kTileIn);
+          tma_load_2d(st + kTileIn, &vmap, &v_full[s], 0, row, pol_v);
+          tma_load_2d(st + kTileIn + 16384, &vmap, &v_full[s], 64, row, pol_v);
         }
       }
     }
@@ -347,6 +351,7 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
       auto pv = [&](int m) {
         if (!mbar_wait(&p_full[m % NP], (m / NP) & 1)) return false;
         if (FP8 && !mbar_wait(v16_full, m & 1)) return false;
+        if (!FP8 && !mbar_wait(&v_full[m % S], (m / S) & 1)) return false;
         tc_fence_after();
         tc_issue_pv<N, FP8>(tmem + kOCol,
                             FP8 ? v16_addr : smem_u32(smem + (m % S) * SM::kStageBytes + kTileIn),
