@@ -864,7 +864,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
             p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
             if (p.fuse_select) seg[q * p.split_keys + (int)(j - k_lo)] = acc[q];
           }
-          hist_inc_warp(hist_s + q * kHistBins, __float_as_uint(acc[q]) >> kHistShift, cand);
+          hist_inc(hist_s + q * kHistBins, __float_as_uint(acc[q]) >> kHistShift, cand);
         }
       }
       asm volatile("bar.sync 2, 128;" ::: "memory");
@@ -1004,20 +1004,16 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         __syncthreads();
         auto val = [&](int e) { return in_smem ? list_s[e] : list_at(e); };
         // level 2: bits [19:9] of the list (every element is in b1)
-        const int m_pad = (m + kThreads - 1) / kThreads * kThreads;
-        for (int e = threadIdx.x; e < m_pad; e += kThreads) {
-          const unsigned v = e < m ? val(e) : 0u;
-          hist_inc_warp(h, (v >> 9) & 2047u, e < m);
-        }
+        for (int e = threadIdx.x; e < m; e += kThreads) hist_inc(h, (val(e) >> 9) & 2047u, true);
         __syncthreads();
         sel_find_bin<kThreads>(h, 2048, s_need[q], s_res, s_tmp);
         const unsigned pre2 = ((unsigned)s_prefix[q] << 11) | (unsigned)s_res[0];
         const int need2 = s_res[1];
         for (int e = threadIdx.x; e < 512; e += kThreads) h[e] = 0u;
         __syncthreads();
-        for (int e = threadIdx.x; e < m_pad; e += kThreads) {
-          const unsigned v = e < m ? val(e) : 0u;
-          hist_inc_warp(h, v & 511u, e < m && (v >> 9) == pre2);
+        for (int e = threadIdx.x; e < m; e += kThreads) {
+          const unsigned v = val(e);
+          hist_inc(h, v & 511u, (v >> 9) == pre2);
         }
         __syncthreads();
         sel_find_bin<kThreads>(h, 512, need2, s_res, s_tmp);
@@ -1270,7 +1266,7 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
         const int t = t0 + q;
         const bool cand = t < p.T && j <= p.L - p.T + t - p.window;
         if (cand) p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
-        hist_inc_warp(hist_s + q * kHistBins, __float_as_uint(acc[q]) >> kHistShift, cand);
+        hist_inc(hist_s + q * kHistBins, __float_as_uint(acc[q]) >> kHistShift, cand);
       }
     }
     softmax_sync<128>();

@@ -495,7 +495,7 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
             const bool cand = key <= i_q - p.window;
             const float v = acc[q][nt][j];
             if (cand) srow[key] = v;
-            hist_inc_warp(hist_s + q * kHistBins, __float_as_uint(v) >> kHistShift, cand, 0xFu);
+            hist_inc(hist_s + q * kHistBins, __float_as_uint(v) >> kHistShift, cand);
           }
       }
     }

@@ -166,12 +166,9 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Histogram increment in shared memory by every lane with `active` (plain
-// atomics: on B200 they beat combining equal bins with __match_any_sync).
-// Every lane of `lanes` calls it.
-__device__ __forceinline__ void hist_inc_warp(unsigned* h, unsigned bin, bool active,
-                                              unsigned lanes = 0xffffffffu) {
-  (void)lanes;
+// Histogram increment in shared memory when `active` (plain atomics: on B200
+// they beat combining equal bins of a warp with __match_any_sync).
+__device__ __forceinline__ void hist_inc(unsigned* h, unsigned bin, bool active) {
   if (active) atomicAdd(h + bin, 1u);
 }
 
