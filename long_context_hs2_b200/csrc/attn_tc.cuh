@@ -99,6 +99,7 @@ struct TcSmem {
 // tile of 128 rows per column half.  E4M3 -> f16 is exact.
 __device__ __forceinline__ void fp8_rows_to_f16(const uint8_t* src, int row0, int nrows,
                                                 int tid, int nthreads, uint8_t* dst) {
+#pragma unroll 4  // independent 16-byte chunks in flight: the loop is latency-bound otherwise
   for (int u = tid; u < nrows * 8; u += nthreads) {
     const int r = row0 + (u >> 3), ch = u & 7;  // codes 16ch .. 16ch+15 of row r
     const uint4 raw = *reinterpret_cast<const uint4*>(src + r * 128 + ((ch ^ (r & 7)) << 4));
@@ -449,18 +450,27 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
 #pragma unroll
       for (int q = 0; q < G; ++q) limit[q] = min(k_hi - 1, p.L - p.T + t0 + q);
       const uint32_t s_addr = tmem + lane_base + s_col(n) + c0;
+      // kHold (NC <= 16): this key's logits of the warp's rows are loaded once and
+      // kept for both sweeps; wider rows reload 16 columns at a time (registers)
+      constexpr bool kHold = NC <= 16;
+      float xs[kHold ? NC : 16];
+      if (kHold) {
+#pragma unroll
+        for (int c = 0; c < NC; c += 16) tmem_ld16(s_addr + c, xs + (c % (kHold ? NC : 16)));
+        tmem_ld_wait();
+      }
       // sweep 1: does any logit exceed its row's reference by more than 2^8?
       bool need = false;
 #pragma unroll
       for (int c = 0; c < NC; c += 16) {
-        float x[16];
-        tmem_ld16(s_addr + c, x);
-        tmem_ld_wait();
+        if (!kHold) {
+          tmem_ld16(s_addr + c, xs);
+          tmem_ld_wait();
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int col = c0 + c + i;
           const bool ok = full_tile || j <= limit[(c + i) / kH + c0 / kH];
-          need |= ok && x[i] * sl > m_ref[col] + kRescaleAbove;
+          need |= ok && xs[(kHold ? c : 0) + i] * sl > m_ref[c0 + c + i] + kRescaleAbove;
         }
       }
       if (n >= NP) {  // the P^T buffer of this tile is free once PV(n - NP) is done
@@ -473,13 +483,14 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
         // new reference: column max of this tile's logits (and the old reference)
 #pragma unroll
         for (int c = 0; c < NC; c += 16) {
-          float x[16];
-          tmem_ld16(s_addr + c, x);
-          tmem_ld_wait();
+          if (!kHold) {
+            tmem_ld16(s_addr + c, xs);
+            tmem_ld_wait();
+          }
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const bool ok = full_tile || j <= limit[(c + i) / kH + c0 / kH];
-            const float v = warp_max(ok ? x[i] * sl : kNegInf);
+            const float v = warp_max(ok ? xs[(kHold ? c : 0) + i] * sl : kNegInf);
             if (lane == 0) tmax[wq * N + c0 + c + i] = v;
           }
         }
@@ -517,6 +528,7 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
             tmem_st16(tmem + lane_base + kOCol + c0 + c, v);
           }
         }
+        tmem_st_wait();  // the rescaled row sums are read back below
       }
       // sweep 2: p = 2^(x - m_ref), row sums, P^T (bf16, or f16 times the
       // value scale for an E4M3 cache) for the PV product; RETAIN: p replaces
@@ -526,15 +538,16 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
         reinterpret_cast<float*>(smem + SM::kMhistOff)[n * N + st] = m_ref[st];
 #pragma unroll
       for (int c = 0; c < NC; c += 16) {
-        float x[16], lv[16], pk[16];
-        tmem_ld16(s_addr + c, x);
+        float lv[16], pk[16];
+        if (!kHold) tmem_ld16(s_addr + c, xs);
         if (RETAIN) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) lv[i] = lreg[(c + i) % (RETAIN ? NC : 1)];
         } else {
           tmem_ld16(tmem + lane_base + 3 * N + c0 + c, lv);
         }
-        tmem_ld_wait();
+        if (!kHold || !RETAIN) tmem_ld_wait();
+        const float* x = xs + (kHold ? c : 0);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int col = c0 + c + i;
