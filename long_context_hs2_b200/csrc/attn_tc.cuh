@@ -430,6 +430,15 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
       for (int c = 0; c < NC; c += 16) tmem_st16(tmem + lane_base + 3 * N + c0 + c, z);
       tmem_st_wait();
     }
+    // E4M3: this key's scales, loaded one tile ahead of their use
+    auto load_scales = [&](int n, float& ks, float& vs) {
+      const long long jn = k_lo + (long long)n * kTcKeys + keyrow;
+      const bool in = FP8 && n < n_tiles && jn < k_hi;
+      ks = in ? p.k_scale[(long long)b * p.L + jn] : 0.f;
+      vs = in ? p.v_scale[(long long)b * p.L + jn] : 0.f;
+    };
+    float ks_next = 0.f, vs_next = 0.f;
+    if (FP8) load_scales(0, ks_next, vs_next);
     for (int n = 0; n < n_tiles; ++n) {
       const int bb = n & 1;
       const long long key0 = k_lo + (long long)n * kTcKeys;
@@ -437,9 +446,9 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
       // this key's logit multiplier and P factor (per-token scales of an E4M3 cache)
       float sl = p.scale_log2, vsc = 1.f;
       if (FP8) {
-        const bool in = j < k_hi;
-        sl *= in ? p.k_scale[(long long)b * p.L + j] : 0.f;
-        vsc = in ? p.v_scale[(long long)b * p.L + j] : 0.f;
+        sl *= ks_next;
+        vsc = vs_next;
+        load_scales(n + 1, ks_next, vs_next);
       }
       failed |= !mbar_wait(&s_full[bb], (n >> 1) & 1);
       tc_fence_after();
@@ -841,11 +850,19 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       const int wq = warp & 3;
       const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
       const int keyrow = wq * 32 + lane;
+      auto load_ks = [&](int n) {
+        const long long jn = k_lo + (long long)n * kTcKeys + keyrow;
+        return (FP8 && !RETAIN && n < n2 && jn < k2_hi) ? p.k_scale[(long long)b * p.L + jn] : 0.f;
+      };
+      float ks_next = load_ks(0);  // E4M3: one tile ahead of its use
       for (int n = 0; n < n2; ++n) {
         const int bb = n & 1;
         const long long j = k_lo + (long long)n * kTcKeys + keyrow;
         float sl = p.scale_log2;
-        if (FP8 && !RETAIN) sl *= j < k2_hi ? p.k_scale[(long long)b * p.L + j] : 0.f;
+        if (FP8 && !RETAIN) {
+          sl *= ks_next;
+          ks_next = load_ks(n + 1);
+        }
         if (!RETAIN && !mbar_wait(&s2_full[bb], (n >> 1) & 1)) break;
         tc_fence_after();
         const uint32_t s_col = RETAIN ? N + n * N : bb * N;
@@ -1252,11 +1269,19 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
     const int wq = warp & 3;
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const int keyrow = wq * 32 + lane;
+    auto load_ks = [&](int n) {
+      const long long jn = k_lo + (long long)n * kTcKeys + keyrow;
+      return (FP8 && n < n_tiles && jn < k_hi) ? p.k_scale[(long long)b * p.L + jn] : 0.f;
+    };
+    float ks_next = load_ks(0);  // E4M3: one tile ahead of its use
     for (int n = 0; n < n_tiles; ++n) {
       const int bb = n & 1;
       const long long j = k_lo + (long long)n * kTcKeys + keyrow;
       float sl = p.scale_log2;
-      if (FP8) sl *= j < k_hi ? p.k_scale[(long long)b * p.L + j] : 0.f;
+      if (FP8) {
+        sl *= ks_next;
+        ks_next = load_ks(n + 1);
+      }
       if (!mbar_wait(&s_full[bb], (n >> 1) & 1)) break;
       tc_fence_after();
       float acc[G];
