@@ -436,8 +436,7 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
     if (st != HS2_OK) return st;
     return run_select(fp, sp, s);
   }
-  if (fp8) return run_full<128, true>(km, vm, fp, pl, sp, s);
-  if (D == 128) return run_full<128, false>(km, vm, fp, pl, sp, s);
+  // head_dim 64 (bf16 only): the mma.sync kernels
   return run_full<64, false>(km, vm, fp, pl, sp, s);
 }
 
