@@ -6,7 +6,9 @@ at 32,768 tokens of bf16 MQA cache, 32 query heads, head_dim 128): the
 full-attention layer with top-1024 + recent-128 selection, then three
 sparse-attention layers that reuse its KV cache and indices, each with its
 own queries.  The metric is hybrid-block decode tokens/s (queries through the
-whole block per second).
+whole block per second).  The same line also carries the KV Bridging GEMM
+("bridge") and the E4M3 configurations ("configs": 4 x 256K decode and the
+4096-query chunk over a 1M-token cache), each timed on its own.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hs2|reference]
 
@@ -45,6 +47,7 @@ def parse():
     ap.add_argument("--impl", choices=["hs2", "reference"], default="hs2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bridge", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
     return ap.parse_args()
 
 
@@ -256,6 +259,84 @@ def bench_bridge(torch, hs2, args, stream):
     return out
 
 
+# ------------------------------------------------------- other configurations --
+def bench_other_configs(torch, hs2, stream, flush_fn, peak_gbs, peak_tflops):
+    """Times the full-attention call and one sparse layer on the E4M3 configurations
+    (4 x 256K decode; the 4096-query chunk over a 1M-token cache), beside the decode
+    metric.  Inputs are drawn on the device in the workloads' distributions (Q, K, V
+    ~ N(0,1); E4M3 codes with the per-token scale max|x|/448); L2 is flushed before
+    every timed call; parity of these shapes is covered by the test suite."""
+    out = {}
+    for name, reps in (("decode_fp8_256k", 10), ("chunk_fp8_1m", 3)):
+        wl = WORKLOADS[name]
+        B, T, L, H, D = wl.B, wl.T, wl.L, wl.H, wl.D
+        g = torch.Generator(device="cuda").manual_seed(wl.seed)
+        q = torch.randn(B, T, H, D, device="cuda", generator=g).to(torch.bfloat16)
+
+        def e4m3(n_rows):
+            x = torch.randn(n_rows, D, device="cuda", generator=g)
+            sc = x.abs().amax(dim=1).clamp_min(1e-30) / 448.0
+            return (x / sc[:, None]).to(torch.float8_e4m3fn).view(torch.uint8), sc
+
+        k, ks = e4m3(B * L)
+        v, vs = e4m3(B * L)
+        kv = hs2.kv_cache(k, v, ks, vs)
+        dt = hs2.HS2_KV_FP8_E4M3
+        slots = wl.topk + wl.window
+        nb = hs2.hs2_full_attn_select_workspace(B, T, L, H, D, wl.topk, wl.window, dt)
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        O = torch.empty(B, T, H, D, device="cuda")
+        idx = torch.empty(B, T, slots, dtype=torch.int32, device="cuda")
+        ns = torch.empty(B, T, dtype=torch.int32, device="cuda")
+
+        def full():
+            hs2.hs2_full_attn_select(q, kv, B, T, L, H, D, wl.scale, wl.topk, wl.window, dt, O,
+                                     None, idx, ns, ws, nb, stream)
+
+        def sparse():
+            hs2.hs2_sparse_attn(q, kv, B, T, L, H, D, wl.scale, idx, ns, slots, dt, O, stream)
+
+        res = {}
+        for label, fn in (("full", full), ("sparse", sparse)):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(reps):
+                flush_fn()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            res[label] = float(np.median(ts))
+        st = hs2.hs2_last_device_status()
+        if st != 0:
+            raise RuntimeError(name + " device status: " + hs2.hs2_status_string(st))
+        kv_bytes = 2 * B * L * (D + 4)
+        sp_bytes = B * T * slots * 2 * (D + 4) + B * T * H * D * 6
+        entry = {"workload": name, "full_ms": res["full"], "sparse_layer_ms": res["sparse"],
+                 "sparse_gbs": sp_bytes / (res["sparse"] * 1e-3) / 1e9,
+                 "sparse_frac_hbm": sp_bytes / (res["sparse"] * 1e-3) / 1e9 / peak_gbs}
+        if T == 1:
+            full_bytes = kv_bytes + B * T * H * D * 6 + B * T * slots * 4
+            entry.update({"full_gbs": full_bytes / (res["full"] * 1e-3) / 1e9,
+                          "full_frac_hbm": full_bytes / (res["full"] * 1e-3) / 1e9 / peak_gbs})
+        else:
+            # causal (query, key, head) triples; QK^T + PV, and the score pass's QK^T again
+            triples = sum((L - T + t + 1) for t in range(T)) * H
+            flops = triples * 4 * D + triples * 2 * D
+            exps = 2 * triples
+            entry.update({"full_tflops": flops / (res["full"] * 1e-3) / 1e12,
+                          "full_frac_tensor": flops / (res["full"] * 1e-3) / 1e12 / peak_tflops,
+                          "full_exp_per_s": exps / (res["full"] * 1e-3)})
+        out[name] = entry
+        del k, v, ks, vs, ws, O, q
+        torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ GPU arm --
 PARTIAL_PROFILE = os.path.join(ROOT, "profiles", "attn_tc_fused_decode_bf16_32k.md")
 KERNEL_SOURCES = ("attn_tc.cuh", "tc_common.cuh", "hs2_common.cuh", "full_attn.cuh", "select.cuh")
@@ -463,6 +544,10 @@ def run_hs2(args, world, rank, local):
                "sample": "one full step: %d sequences x 1 query, full attention + selection + "
                          "%d sparse layers (%.1f s)" % (B, wl.n_sparse, dts)}
     bridge = bench_bridge(torch, hs2, args, stream) if (rank == 0 and not args.no_bridge) else None
+    others = None
+    if rank == 0 and not args.no_configs:
+        others = bench_other_configs(torch, hs2, stream, l2_flush, peak,
+                                     measured_tensor_peak()[0])
     del g_full, g_sparse
     if world > 1:
         dist.barrier()
@@ -504,6 +589,7 @@ def run_hs2(args, world, rank, local):
         "clocks": clk,
         "cpu_baseline": cpu,
         "bridge": bridge,
+        "configs": others,
     }
     print(json.dumps(line), flush=True)
 
