@@ -300,8 +300,13 @@ hs2_status run_sparse(const SparseParams& p, cudaStream_t s) {
   using SM = SparseSmem<MT, D, FP8>;
   auto k = sparse_attn_kernel<MT, D, FP8>;
   if (!set_smem(k, SM::kBytes)) return HS2_ERR_CUDA;
-  return launch_ex(k, dim3((unsigned)((long long)p.B * p.T * p.cs)), dim3(128), SM::kBytes, s,
-                   p.cs, false, true, p);
+  // the position array holds this launch's largest per-CTA share of the slots
+  // (rank 0's), plus n_sel: small slot counts let two CTAs share an SM
+  const int tiles_max = (p.slots + kSpTile - 1) / kSpTile;
+  const int my_max = (tiles_max + p.cs - 1) / p.cs;
+  const size_t bytes = (size_t)SM::kPosOff + (size_t)(my_max * kSpTile + 4) * 4 + 1024;
+  return launch_ex(k, dim3((unsigned)((long long)p.B * p.T * p.cs)), dim3(128), bytes, s, p.cs,
+                   false, true, p);
 }
 
 }  // namespace
