@@ -24,8 +24,13 @@
 // as f16: exact for bf16 values of magnitude >= 2^-14, and P is written as
 // f16).  The per-token scales need no extra pass: the thread that owns key j
 // multiplies its logits by k_scale[j] and its P values by v_scale[j].
-//   attn_tc_partial : per (group, split): reference max m, sum l and
-//                     un-normalised O of the split.
+//   attn_tc_fused   : decode shapes (32 rows per group): the partial pass of
+//                     a (group, split), a group barrier, the score pass over
+//                     the same split (from logits kept in TMEM when the split
+//                     has at most 15 tiles, else recomputed from K), and the
+//                     group's top-k selection -- one cooperative launch.
+//   attn_tc_partial : other shapes, per (group, split): reference max m, sum
+//                     l and un-normalised O of the split.
 //   attn_tc_score   : merges the splits into lse and O, then recomputes S^T per
 //                     tile and writes score_j = sum over a query's heads of
 //                     exp(s - lse), with the level-1 selection histogram.
