@@ -103,8 +103,13 @@ def _check(fn: str, st: int):
 
 
 def kv_cache(k, v, k_scale=None, v_scale=None) -> hs2_kv_cache:
-    """The C struct of one layer's cache from device tensors (or raw pointers)."""
-    return hs2_kv_cache(_ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale))
+    """The C struct of one layer's cache from device tensors (or raw pointers).
+    The struct holds references to the tensors it was made from, so that their
+    memory stays allocated for as long as the struct (or a CUDA graph that
+    captured calls with it, while the caller keeps the struct) is in use."""
+    c = hs2_kv_cache(_ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale))
+    c._tensors = (k, v, k_scale, v_scale)
+    return c
 
 
 def hs2_version() -> int:

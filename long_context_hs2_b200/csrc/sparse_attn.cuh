@@ -9,7 +9,9 @@
 // query's tiles in flight at once), runs the warp attention core (warps split
 // every tile's keys 4 ways) and merges its warps.  Then every CTA of the
 // cluster merges one slice of the query's H x D output from all CTAs'
-// partials, read through distributed shared memory.  No global scratch is
+// partials.  Each CTA pushes the slices of its merged partial to the CTAs that
+// own them with distributed-shared-memory stores; one cluster barrier later
+// every CTA merges its slice from its own shared memory.  No global scratch is
 // needed.
 #pragma once
 
@@ -59,26 +61,37 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
+// Cluster barrier halves.  Every thread of every CTA of the cluster arrives
+// once per phase; the wait ends when all have arrived.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float2 ld_dsmem_f32x2(uint32_t addr) {
-  float2 v;
-  asm("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
+__device__ __forceinline__ void st_dsmem_f32x2(uint32_t addr, float2 v) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y)
+               : "memory");
 }
-__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
-  float4 v;
-  asm("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-      : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-      : "r"(addr));
-  return v;
+__device__ __forceinline__ void st_dsmem_f32x4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
+// 4-byte global->shared copy (the L1-allocating form; the .cg form moves 16
+// bytes only); src_bytes == 0 writes zeros.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
 }
 
 // Gathers the K/V rows of one 64-slot tile (positions pos[0..63], -1 =
@@ -114,13 +127,18 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   uint8_t* smem = align1024(smem_raw);
   uint8_t* qs = smem + SM::kQOff;
   float2* ml_s = reinterpret_cast<float2*>(smem + SM::kMlOff);
+  // merge inputs: with a cluster, [source CTA][row of this CTA's slice] (m, l)
+  // and [source CTA][element of the slice] O, written by the cluster's CTAs
   float2* cl_ml = reinterpret_cast<float2*>(smem + SM::kClOff);
   float* cl_o = reinterpret_cast<float*>(smem + SM::kClOff + SM::kRowsQ * 8);
   int* pos_all = reinterpret_cast<int*>(smem + SM::kPosOff);  // [my_tiles][64]
 
-  pdl_launch_dependents();
-  pdl_wait();  // indices, counts and queries come from earlier kernels
   const int cs = p.cs;
+  pdl_launch_dependents();
+  // first cluster phase: this CTA runs (its merge inputs may be written once
+  // the phase completes, just before the merge)
+  if (cs > 1) cluster_arrive_relaxed();
+  pdl_wait();  // indices, counts and queries come from earlier kernels
   const uint32_t rank = cs > 1 ? cluster_ctarank() : 0u;
   const long long qrow = blockIdx.x / cs;  // b*T + t
   const int b = (int)(qrow / p.T);
@@ -130,24 +148,28 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   // tiles of this CTA if every slot were used: tile k of the CTA is slot tile rank + k*cs
   const int tiles_max = (p.slots + kSpTile - 1) / kSpTile;
   const int my_max = tiles_max > (int)rank ? (tiles_max - (int)rank + cs - 1) / cs : 0;
-  // positions of this CTA's slots, loaded together with n_sel (no dependent round trip)
+  // positions of this CTA's slots, n_sel and the query rows (head h = row;
+  // rows >= H are zero) in one asynchronous round trip; slots past `slots`
+  // read as 0 and are masked below (they lie past n_sel)
   int* nsel_s = pos_all + my_max * kSpTile;
-  if (threadIdx.x == 0) *nsel_s = p.n_sel[qrow];
+  if (threadIdx.x == 0) cp_async4(smem_u32(nsel_s), p.n_sel + qrow, 4);
   for (int u = threadIdx.x; u < my_max * kSpTile; u += 128) {
     const int slot = ((int)rank + (u / kSpTile) * cs) * kSpTile + (u % kSpTile);
-    pos_all[u] = slot < p.slots ? sel[slot] : -1;
+    const bool in = slot < p.slots;
+    cp_async4(smem_u32(pos_all + u), in ? sel + slot : sel, in ? 4 : 0);
   }
-
-  // query rows: head h = row (rows >= H are zero)
   {
     constexpr int kChunks = D * 2 / 16;
+    const uint32_t q_s = smem_u32(qs);
     for (int u = threadIdx.x; u < SM::kRowsQ * kChunks; u += 128) {
       const int r = u / kChunks, ch = u % kChunks;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < p.H) v = *reinterpret_cast<const uint4*>(p.q + (qrow * p.H + r) * D + ch * 8);
-      *reinterpret_cast<uint4*>(qs + sw128_offset(r, ch * 16, SM::kRowsQ)) = v;
+      const bool in = r < p.H;
+      cp_async16(q_s + sw128_offset(r, ch * 16, SM::kRowsQ),
+                 p.q + (qrow * p.H + (in ? r : 0)) * D + ch * 8, in ? 16 : 0);
     }
   }
+  cp_async_commit();
+  cp_async_wait<0>();
   const float* ksc = FP8 ? p.k_scale + (long long)b * p.L : nullptr;
   const float* vsc = FP8 ? p.v_scale + (long long)b * p.L : nullptr;
 
@@ -236,7 +258,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   cp_async_wait<0>();
   __syncthreads();
 
-  // merge the warps into this CTA's (m, l, O) in cl_ml / cl_o
+  // merge the warps: rescale each warp's O to the CTA's row maximum
   float lf[MT][2], f[MT][2];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
@@ -258,15 +280,16 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
     }
   float* obuf = reinterpret_cast<float*>(smem);
   warp_store_o<MT, D>(st, f, obuf + warp * SM::kRowsQ * (D + 8));
+  // CTA `rank` of the cluster owns rows [rank*rpc, (rank+1)*rpc) of the H x D
+  // output (H / cs is a whole number: H in {8, 16, 32}, cs in {1, 2, 4, 8})
+  const int rpc = p.H / cs;
+  const int chunk = rpc * D;
+  const uint32_t ml_addr = smem_u32(cl_ml), o_addr = smem_u32(cl_o);
+  if (cs > 1) cluster_wait_acquire();  // first phase: every CTA of the cluster runs
   __syncthreads();
-  for (int u = threadIdx.x; u < SM::kRowsQ * D; u += 128) {
-    const int r = u / D, d = u % D;
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < kSpWarps; ++w) acc += obuf[(w * SM::kRowsQ + r) * (D + 8) + d];
-    cl_o[u] = acc;
-  }
-  if (threadIdx.x < SM::kRowsQ) {
+  // this CTA's (m, l) per row and its O summed over the warps, stored locally
+  // (no cluster) or pushed to the slice's owner
+  if (threadIdx.x < p.H) {
     const int r = threadIdx.x;
     float M = kNegInf;
     for (int w = 0; w < kSpWarps; ++w) M = fmaxf(M, ml_s[w * SM::kRowsQ + r].x);
@@ -276,49 +299,64 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
         const float2 v = ml_s[w * SM::kRowsQ + r];
         lt += v.y * fast_exp2(v.x - M);
       }
-    cl_ml[r] = make_float2(M, lt);
+    if (cs == 1)
+      cl_ml[r] = make_float2(M, lt);
+    else
+      st_dsmem_f32x2(mapa_shared(ml_addr + ((int)rank * rpc + r % rpc) * 8, (uint32_t)(r / rpc)),
+                     make_float2(M, lt));
+  }
+  for (int u = 4 * threadIdx.x; u < p.H * D; u += 4 * 128) {
+    const int r = u / D, d = u % D;
+    float4 acc = *reinterpret_cast<const float4*>(obuf + r * (D + 8) + d);
+#pragma unroll
+    for (int w = 1; w < kSpWarps; ++w) {
+      const float4 o = *reinterpret_cast<const float4*>(obuf + (w * SM::kRowsQ + r) * (D + 8) + d);
+      acc.x += o.x;
+      acc.y += o.y;
+      acc.z += o.z;
+      acc.w += o.w;
+    }
+    if (cs == 1)
+      *reinterpret_cast<float4*>(cl_o + u) = acc;
+    else
+      st_dsmem_f32x4(mapa_shared(o_addr + ((int)rank * chunk + u % chunk) * 4, (uint32_t)(u / chunk)),
+                     acc);
   }
   if (cs == 1) {
     __syncthreads();
-    for (int u = threadIdx.x; u < p.H * D; u += 128) {
+    for (int u = 4 * threadIdx.x; u < p.H * D; u += 4 * 128) {
       const float2 v = cl_ml[u / D];
-      p.o[qrow * p.H * D + u] = v.y > 0.f ? cl_o[u] / v.y : 0.f;
+      const float inv = v.y > 0.f ? 1.f / v.y : 0.f;
+      const float4 o = *reinterpret_cast<const float4*>(cl_o + u);
+      *reinterpret_cast<float4*>(p.o + qrow * p.H * D + u) =
+          make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
     }
     return;
   }
-  cluster_sync_all();
-  // CTA `rank` merges elements [rank*chunk, (rank+1)*chunk) of the H x D output
-  // (chunk is a multiple of 4: H*D is a multiple of 512 and cs <= 8)
-  const int chunk = p.H * D / cs;
-  const uint32_t ml_addr = smem_u32(cl_ml), o_addr = smem_u32(cl_o);
-  for (int u = (int)rank * chunk + 4 * threadIdx.x; u < ((int)rank + 1) * chunk; u += 4 * 128) {
-    const int r = u / D;
-    float2 mls[8];
+  // second phase: every CTA's pushes have landed; nothing reads another CTA's
+  // shared memory after it, so each CTA may exit when its slice is written
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  for (int e = 4 * threadIdx.x; e < chunk; e += 4 * 128) {
+    const int rl = e / D;
     float M = kNegInf;
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (q < cs) {
-        mls[q] = ld_dsmem_f32x2(mapa_shared(ml_addr + r * 8, q));
-        M = fmaxf(M, mls[q].x);
-      }
+    for (int q = 0; q < cs; ++q) M = fmaxf(M, cl_ml[q * rpc + rl].x);
     float lt = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (q < cs) {
-        const float4 o = ld_dsmem_f32x4(mapa_shared(o_addr + u * 4, q));
-        const float f = (M == kNegInf || mls[q].x == kNegInf) ? 0.f : fast_exp2(mls[q].x - M);
-        lt += mls[q].y * f;
-        acc.x += f * o.x;
-        acc.y += f * o.y;
-        acc.z += f * o.z;
-        acc.w += f * o.w;
-      }
+    for (int q = 0; q < cs; ++q) {
+      const float2 ml = cl_ml[q * rpc + rl];
+      const float f = (M == kNegInf || ml.x == kNegInf) ? 0.f : fast_exp2(ml.x - M);
+      const float4 o = *reinterpret_cast<const float4*>(cl_o + q * chunk + e);
+      lt += ml.y * f;
+      acc.x += f * o.x;
+      acc.y += f * o.y;
+      acc.z += f * o.z;
+      acc.w += f * o.w;
+    }
     const float inv = lt > 0.f ? 1.f / lt : 0.f;
-    *reinterpret_cast<float4*>(p.o + qrow * p.H * D + u) =
+    *reinterpret_cast<float4*>(p.o + qrow * p.H * D + (long long)rank * chunk + e) =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   }
-  cluster_sync_all();  // keep every CTA's shared memory alive until all reads are done
 }
 
 }  // namespace hs2

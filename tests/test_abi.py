@@ -98,6 +98,23 @@ def test_stage_events_pairing(lib):
     assert lib.hs2_set_stage_events(None, None) == 0
 
 
+def test_kv_cache_keeps_its_tensors():
+    # the struct holds raw pointers; it must keep the tensors behind them alive
+    import gc
+    import weakref
+    import torch
+    k, v = torch.zeros(8), torch.zeros(8)
+    rk = weakref.ref(k)
+    c = hs2.kv_cache(k, v)
+    ptr = k.data_ptr()
+    del k, v
+    gc.collect()
+    assert rk() is not None and c.k == ptr
+    del c
+    gc.collect()
+    assert rk() is None
+
+
 def test_product_path_does_not_import_oracle():
     pkg = os.path.join(ROOT, "long_context_hs2_b200")
     for dirpath, _, files in os.walk(pkg):
