@@ -300,13 +300,11 @@ hs2_status run_sparse(const SparseParams& p, cudaStream_t s) {
   using SM = SparseSmem<MT, D, FP8>;
   auto k = sparse_attn_kernel<MT, D, FP8>;
   if (!set_smem(k, SM::kBytes)) return HS2_ERR_CUDA;
-  // the position array holds this launch's largest per-CTA share of the slots
-  // (rank 0's), plus n_sel: small slot counts let two CTAs share an SM
-  const int tiles_max = (p.slots + kSpTile - 1) / kSpTile;
-  const int my_max = (tiles_max + p.cs - 1) / p.cs;
-  const size_t bytes = (size_t)SM::kPosOff + (size_t)(my_max * kSpTile + 4) * 4 + 1024;
-  return launch_ex(k, dim3((unsigned)((long long)p.B * p.T * p.cs)), dim3(128), bytes, s, p.cs,
-                   false, true, p);
+  // the position array holds one CTA's share of the slots in whole tiles, plus n_sel
+  const int tiles_max = (sparse_share(p.slots, p.cs) + kSpTile - 1) / kSpTile;
+  const size_t bytes = (size_t)SM::kPosOff + (size_t)(tiles_max * kSpTile + 4) * 4 + 1024;
+  return launch_ex(k, dim3((unsigned)((long long)p.B * p.T * p.cs)), dim3(kSpThreads), bytes, s,
+                   p.cs, false, true, p);
 }
 
 }  // namespace

@@ -1,26 +1,29 @@
 // Sparse-attention layer with KV Reuse: each query attends over its selected
 // positions of the shared cache.
 //
-// One thread-block cluster of CS CTAs per query.  The query's selected slots
-// are cut into 64-slot tiles dealt round-robin to the cluster's CTAs; each CTA
-// loads (and range-checks) its slots' positions together with the query's
-// n_sel, gathers its tiles' K/V rows with 16-byte cp.async copies into
-// 128B-swizzled shared-memory tiles (a multi-stage ring, all of a decode
-// query's tiles in flight at once), runs the warp attention core (warps split
-// every tile's keys 4 ways) and merges its warps.  Then every CTA of the
-// cluster merges one slice of the query's H x D output from all CTAs'
-// partials.  Each CTA pushes the slices of its merged partial to the CTAs that
-// own them with distributed-shared-memory stores; one cluster barrier later
-// every CTA merges its slice from its own shared memory.  No global scratch is
-// needed.
+// One thread-block cluster of CS CTAs per query.  CTA r of the cluster takes
+// the contiguous slot range [r*S, (r+1)*S), S = ceil(slots / CS), so every CTA
+// of a full selection has the same work.  It loads its slots' positions, the
+// query's n_sel and the query rows in one asynchronous round trip,
+// range-checks the positions, and walks its range in 128-slot tiles: the K/V
+// rows of a tile are gathered with 16-byte cp.async copies into 128B-swizzled
+// shared-memory tiles (a two-stage ring) and each of the 8 warps runs the
+// warp attention core over its 16-key group of the tile (a group with no
+// valid key is neither gathered nor computed).  The CTA merges its warps;
+// then each CTA pushes the slices of its merged partial to the CTAs that own
+// them with distributed-shared-memory stores, and one cluster barrier later
+// every CTA merges its slice of the query's H x D output from its own shared
+// memory.  No global scratch is needed.
 #pragma once
 
 #include "attn_warp.cuh"
 
 namespace hs2 {
 
-constexpr int kSpTile = 64;
-constexpr int kSpWarps = 4;
+constexpr int kSpWarps = 8;
+constexpr int kSpThreads = kSpWarps * 32;
+constexpr int kSpGroup = 16;                   // keys per warp per tile
+constexpr int kSpTile = kSpWarps * kSpGroup;   // keys per tile
 
 struct SparseParams {
   const __nv_bfloat16* q;  // [B][T][H][D]
@@ -36,24 +39,29 @@ struct SparseParams {
   float scale_log2;
 };
 
+// Slots per CTA of a cluster of cs CTAs.
+__host__ __device__ __forceinline__ int sparse_share(int slots, int cs) {
+  return (slots + cs - 1) / cs;
+}
+
 template <int MT, int D, bool FP8>
 struct SparseSmem {
   static constexpr int kRowsQ = MT * 16;
   static constexpr int kElem = FP8 ? 1 : 2;
   static constexpr int kTileBytes = kSpTile * D * kElem;
-  static constexpr int kStages = 3;
+  static constexpr int kStages = 2;
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStagingBytes = FP8 ? kSpWarps * 2 * 16 * D * 2 : 0;
+  static constexpr int kStagingBytes = FP8 ? kSpWarps * 2 * kSpGroup * D * 2 : 0;
   static constexpr int kObufBytes = kSpWarps * kRowsQ * (D + 8) * 4;
   static constexpr int kRing = kStages * kStageBytes + kStagingBytes;
   static constexpr int kMain = kRing > kObufBytes ? kRing : kObufBytes;
   static constexpr int kQOff = kMain;
   static constexpr int kMlOff = kQOff + kRowsQ * D * 2;
-  static constexpr int kClOff = kMlOff + kSpWarps * kRowsQ * 8;  // CTA result: ml[rows], o[rows][D]
+  static constexpr int kClOff = kMlOff + kSpWarps * kRowsQ * 8;  // merge inputs
   static constexpr int kClBytes = kRowsQ * 8 + kRowsQ * D * 4;
   static constexpr int kPosOff = kClOff + kClBytes;               // positions of the CTA's slots
   static constexpr int kMaxSlots = 4096;
-  static constexpr int kBytes = kPosOff + (kMaxSlots + 64 + 4) * 4 + 1024;
+  static constexpr int kBytes = kPosOff + (kMaxSlots + kSpTile + 4) * 4 + 1024;
 };
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -94,34 +102,33 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, int src
                : "memory");
 }
 
-// Gathers the K/V rows of one 64-slot tile (positions pos[0..63], -1 =
-// masked) into a ring stage.  All 128 threads; one commit group.
+// Gathers the K/V rows 0 .. rows-1 of one tile (positions pos[r], -1 =
+// masked: zero-filled) into a ring stage.  All threads; one commit group.
 template <int D, bool FP8>
 __device__ __forceinline__ void sparse_gather_tile(const SparseParams& p, int b, const int* pos,
-                                                   uint8_t* stage) {
+                                                   int rows, uint8_t* stage) {
   constexpr int kRowBytes = D * (FP8 ? 1 : 2);
   constexpr int kChunks = kRowBytes / 16;
   constexpr int kTileBytes = kSpTile * kRowBytes;
   const uint32_t dst0 = smem_u32(stage);
-  for (int u = threadIdx.x; u < 2 * kSpTile * kChunks; u += kSpWarps * 32) {
-    const int tsr = u / (kSpTile * kChunks);  // 0: K, 1: V
-    const int rem = u % (kSpTile * kChunks);
-    const int r = rem / kChunks, ch = rem % kChunks;
+  const long long row0 = (long long)b * p.L;
+  for (int u = threadIdx.x; u < rows * kChunks; u += kSpThreads) {
+    const int r = u / kChunks, ch = u % kChunks;
     const int ps = pos[r];
-    const uint8_t* base = tsr ? p.v : p.k;
-    const uint8_t* src = base + ((long long)b * p.L + (ps < 0 ? 0 : ps)) * kRowBytes + ch * 16;
+    const long long src_off = (row0 + (ps < 0 ? 0 : ps)) * kRowBytes + ch * 16;
     uint32_t off;
     if (FP8)
       off = (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
     else
       off = sw128_offset(r, ch * 16, kSpTile);
-    cp_async16(dst0 + tsr * kTileBytes + off, src, ps < 0 ? 0 : 16);
+    cp_async16(dst0 + off, p.k + src_off, ps < 0 ? 0 : 16);
+    cp_async16(dst0 + kTileBytes + off, p.v + src_off, ps < 0 ? 0 : 16);
   }
   cp_async_commit();
 }
 
 template <int MT, int D, bool FP8>
-__global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) {
+__global__ void __launch_bounds__(kSpThreads) sparse_attn_kernel(const SparseParams p) {
   using SM = SparseSmem<MT, D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -131,7 +138,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   // and [source CTA][element of the slice] O, written by the cluster's CTAs
   float2* cl_ml = reinterpret_cast<float2*>(smem + SM::kClOff);
   float* cl_o = reinterpret_cast<float*>(smem + SM::kClOff + SM::kRowsQ * 8);
-  int* pos_all = reinterpret_cast<int*>(smem + SM::kPosOff);  // [my_tiles][64]
+  int* pos_all = reinterpret_cast<int*>(smem + SM::kPosOff);  // [tiles][kSpTile]
 
   const int cs = p.cs;
   pdl_launch_dependents();
@@ -145,23 +152,25 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int32_t* sel = p.idx + qrow * p.slots;
-  // tiles of this CTA if every slot were used: tile k of the CTA is slot tile rank + k*cs
-  const int tiles_max = (p.slots + kSpTile - 1) / kSpTile;
-  const int my_max = tiles_max > (int)rank ? (tiles_max - (int)rank + cs - 1) / cs : 0;
-  // positions of this CTA's slots, n_sel and the query rows (head h = row;
-  // rows >= H are zero) in one asynchronous round trip; slots past `slots`
-  // read as 0 and are masked below (they lie past n_sel)
-  int* nsel_s = pos_all + my_max * kSpTile;
+  // this CTA's slot range [lo, hi) and the tiles it would take if all were used
+  const int share = sparse_share(p.slots, cs);
+  const int lo = (int)rank * share;
+  const int hi = min(lo + share, p.slots);
+  const int tiles_max = (share + kSpTile - 1) / kSpTile;
+  // positions of the range, n_sel and the query rows (head h = row; rows >= H
+  // are zero) in one asynchronous round trip; slots past the range read as 0
+  // and are masked below
+  int* nsel_s = pos_all + tiles_max * kSpTile;
   if (threadIdx.x == 0) cp_async4(smem_u32(nsel_s), p.n_sel + qrow, 4);
-  for (int u = threadIdx.x; u < my_max * kSpTile; u += 128) {
-    const int slot = ((int)rank + (u / kSpTile) * cs) * kSpTile + (u % kSpTile);
-    const bool in = slot < p.slots;
+  for (int u = threadIdx.x; u < tiles_max * kSpTile; u += kSpThreads) {
+    const int slot = lo + u;
+    const bool in = slot < hi;
     cp_async4(smem_u32(pos_all + u), in ? sel + slot : sel, in ? 4 : 0);
   }
   {
     constexpr int kChunks = D * 2 / 16;
     const uint32_t q_s = smem_u32(qs);
-    for (int u = threadIdx.x; u < SM::kRowsQ * kChunks; u += 128) {
+    for (int u = threadIdx.x; u < SM::kRowsQ * kChunks; u += kSpThreads) {
       const int r = u / kChunks, ch = u % kChunks;
       const bool in = r < p.H;
       cp_async16(q_s + sw128_offset(r, ch * 16, SM::kRowsQ),
@@ -175,13 +184,13 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
 
   __syncthreads();
   const int n = max(0, min(*nsel_s, p.slots));
-  const int n_tiles_all = (n + kSpTile - 1) / kSpTile;
-  const int my_tiles = n_tiles_all > (int)rank ? (n_tiles_all - (int)rank + cs - 1) / cs : 0;
-  // mask slots past n_sel; range-check the others
-  for (int u = threadIdx.x; u < my_tiles * kSpTile; u += 128) {
-    const int slot = ((int)rank + (u / kSpTile) * cs) * kSpTile + (u % kSpTile);
+  const int end = min(hi, n);                  // valid slots: [lo, end)
+  const int n_valid = max(0, end - lo);
+  const int my_tiles = (n_valid + kSpTile - 1) / kSpTile;
+  // mask slots past n_sel or past the range; range-check the others
+  for (int u = threadIdx.x; u < my_tiles * kSpTile; u += kSpThreads) {
     int ps = pos_all[u];
-    if (slot >= n) {
+    if (u >= n_valid) {
       ps = -1;
     } else if (ps < 0 || (long long)ps >= p.L) {
       raise_status(kStatusBadIndex);
@@ -190,12 +199,18 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
     pos_all[u] = ps;
   }
   __syncthreads();
+  // rows of tile k that hold a valid slot's group: whole 16-key groups
+  auto tile_rows = [&](int k) {
+    const int v = min(kSpTile, n_valid - k * kSpTile);
+    return (v + kSpGroup - 1) / kSpGroup * kSpGroup;
+  };
 
   // prologue: fill kStages-1 ring slots
 #pragma unroll
   for (int s = 0; s < SM::kStages - 1; ++s) {
     if (s < my_tiles)
-      sparse_gather_tile<D, FP8>(p, b, pos_all + s * kSpTile, smem + s * SM::kStageBytes);
+      sparse_gather_tile<D, FP8>(p, b, pos_all + s * kSpTile, tile_rows(s),
+                                 smem + s * SM::kStageBytes);
     else
       cp_async_commit();
   }
@@ -203,57 +218,62 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   WarpAttn<MT, D> st;
   st.init();
   const uint32_t q_base = smem_u32(qs);
-  uint8_t* stg_k = smem + SM::kStages * SM::kStageBytes + warp * 2 * 16 * D * 2;
-  uint8_t* stg_v = stg_k + 16 * D * 2;
+  uint8_t* stg_k = smem + SM::kStages * SM::kStageBytes + warp * 2 * kSpGroup * D * 2;
+  uint8_t* stg_v = stg_k + kSpGroup * D * 2;
 
   for (int k = 0; k < my_tiles; ++k) {
     {  // refill the slot consumed in step k-1 (all threads passed the barrier ending it)
       const int kn = k + SM::kStages - 1;
       if (kn < my_tiles)
-        sparse_gather_tile<D, FP8>(p, b, pos_all + kn * kSpTile,
+        sparse_gather_tile<D, FP8>(p, b, pos_all + kn * kSpTile, tile_rows(kn),
                                    smem + (kn % SM::kStages) * SM::kStageBytes);
       else
         cp_async_commit();
     }
     cp_async_wait<SM::kStages - 1>();  // tile k has landed
     __syncthreads();
-    const int s = k % SM::kStages;
-    uint8_t* stage = smem + s * SM::kStageBytes;
-    const int* pos = pos_all + k * kSpTile;
-    uint32_t kt, vt;
-    int key0, rows;
-    if (FP8) {
-      warp_fp8_rows_to_bf16(stage, warp * 16, 16, stg_k, 16);
-      warp_fp8_rows_to_bf16(stage + SM::kTileBytes, warp * 16, 16, stg_v, 16);
-      __syncwarp();
-      kt = smem_u32(stg_k);
-      vt = smem_u32(stg_v);
-      key0 = 0;
-      rows = 16;
-    } else {
-      kt = smem_u32(stage);
-      vt = smem_u32(stage + SM::kTileBytes);
-      key0 = warp * 16;
-      rows = kSpTile;
-    }
-    float x[MT][2][4];
-    warp_qk<MT, D>(q_base, kt, key0, rows, x);
-    float pvs[2][2];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int ps = pos[warp * 16 + nt * 8 + 2 * c + j];
-        const float ks = (FP8 && ps >= 0) ? ksc[ps] : 1.f;
-        pvs[nt][j] = (FP8 && ps >= 0) ? vsc[ps] : 1.f;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            x[mt][nt][2 * h + j] = ps >= 0 ? x[mt][nt][2 * h + j] * (p.scale_log2 * ks) : kNegInf;
+    // this warp's 16-key group: skipped when it holds no valid slot (its rows
+    // were not gathered)
+    if (warp * kSpGroup < tile_rows(k)) {
+      const int s = k % SM::kStages;
+      uint8_t* stage = smem + s * SM::kStageBytes;
+      const int* pos = pos_all + k * kSpTile;
+      uint32_t kt, vt;
+      int key0, rows;
+      if (FP8) {
+        warp_fp8_rows_to_bf16(stage, warp * kSpGroup, kSpGroup, stg_k, kSpGroup);
+        warp_fp8_rows_to_bf16(stage + SM::kTileBytes, warp * kSpGroup, kSpGroup, stg_v, kSpGroup);
+        __syncwarp();
+        kt = smem_u32(stg_k);
+        vt = smem_u32(stg_v);
+        key0 = 0;
+        rows = kSpGroup;
+      } else {
+        kt = smem_u32(stage);
+        vt = smem_u32(stage + SM::kTileBytes);
+        key0 = warp * kSpGroup;
+        rows = kSpTile;
       }
-    warp_softmax_pv<MT, D>(st, x, vt, key0, rows, pvs);
-    __syncthreads();  // ring slot s is free again
+      float x[MT][2][4];
+      warp_qk<MT, D>(q_base, kt, key0, rows, x);
+      float pvs[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int ps = pos[warp * kSpGroup + nt * 8 + 2 * c + j];
+          const float ks = (FP8 && ps >= 0) ? ksc[ps] : 1.f;
+          pvs[nt][j] = (FP8 && ps >= 0) ? vsc[ps] : 1.f;
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              x[mt][nt][2 * h + j] =
+                  ps >= 0 ? x[mt][nt][2 * h + j] * (p.scale_log2 * ks) : kNegInf;
+        }
+      warp_softmax_pv<MT, D>(st, x, vt, key0, rows, pvs);
+    }
+    __syncthreads();  // ring slot k % kStages is free again
   }
   cp_async_wait<0>();
   __syncthreads();
@@ -305,7 +325,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
       st_dsmem_f32x2(mapa_shared(ml_addr + ((int)rank * rpc + r % rpc) * 8, (uint32_t)(r / rpc)),
                      make_float2(M, lt));
   }
-  for (int u = 4 * threadIdx.x; u < p.H * D; u += 4 * 128) {
+  for (int u = 4 * threadIdx.x; u < p.H * D; u += 4 * kSpThreads) {
     const int r = u / D, d = u % D;
     float4 acc = *reinterpret_cast<const float4*>(obuf + r * (D + 8) + d);
 #pragma unroll
@@ -324,7 +344,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   }
   if (cs == 1) {
     __syncthreads();
-    for (int u = 4 * threadIdx.x; u < p.H * D; u += 4 * 128) {
+    for (int u = 4 * threadIdx.x; u < p.H * D; u += 4 * kSpThreads) {
       const float2 v = cl_ml[u / D];
       const float inv = v.y > 0.f ? 1.f / v.y : 0.f;
       const float4 o = *reinterpret_cast<const float4*>(cl_o + u);
@@ -337,7 +357,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(const SparseParams p) 
   // shared memory after it, so each CTA may exit when its slice is written
   cluster_arrive_release();
   cluster_wait_acquire();
-  for (int e = 4 * threadIdx.x; e < chunk; e += 4 * 128) {
+  for (int e = 4 * threadIdx.x; e < chunk; e += 4 * kSpThreads) {
     const int rl = e / D;
     float M = kNegInf;
     for (int q = 0; q < cs; ++q) M = fmaxf(M, cl_ml[q * rpc + rl].x);
