@@ -188,3 +188,10 @@ def test_decode_bf16_64k_many_tiles_per_split():
     # 29 key tiles per split: more than tensor memory keeps, so the fused
     # kernel's score pass recomputes the logits from K (bf16 cache)
     _check_block(WORKLOADS["decode_bf16_32k"].resized(L=65536, n_needles=32), sparse_layers=[0])
+
+
+def test_decode_bf16_unaligned_slot_shares():
+    # 1000 + 100 slots over a cluster of 8 CTAs: each CTA's 138-slot share
+    # starts inside a 16-key group and ends on a partly valid one
+    _check_block(WORKLOADS["decode_bf16_32k"].resized(L=8192, topk=1000, window=100,
+                                                      n_needles=16))
