@@ -37,6 +37,11 @@ MUTANTS = {
     "sparse_uses_v_as_k": ("kd[(size_t)n * D + d] = kv.key(b, sel[n], d);", "kd[(size_t)n * D + d] = kv.val(b, sel[n], d);"),
     "sparse_softmax_not_normalised": ("for (int n = 0; n < ns; ++n) pr[n] = std::exp(pr[n] - m) / l;",
                                       "for (int n = 0; n < ns; ++n) pr[n] = std::exp(pr[n] - m);"),
+    "sparse_scale_dropped": ("pr[n] = scale * acc;", "pr[n] = acc;"),
+    "sparse_normaliser_drops_last_key": ("for (int n = 0; n < ns; ++n) l += std::exp(pr[n] - m);",
+                                         "for (int n = 0; n + 1 < ns; ++n) l += std::exp(pr[n] - m);"),
+    "output_uses_next_heads_p": ("for (int d = 0; d < D; ++d) acc[h * D + d] += pj * vj[d];",
+                                 "for (int d = 0; d < D; ++d) acc[h * D + d] += p[(size_t)((h + 1) % H) * n + j] * vj[d];"),
     "fp8_value_scale_ignored": ("if (fp8) return e4m3_to_f64(((const uint8_t*)base)[off]) * (double)sc[(int64_t)b * L + j];",
                                 "if (fp8) return e4m3_to_f64(((const uint8_t*)base)[off]) * (double)sc[(int64_t)b * L];"),
 }
