@@ -82,3 +82,17 @@ def test_two_rank_replicas_timing_and_reference_arm():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["metric"] == "hybrid-block decode tokens/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_profiled_traffic_follows_the_kernel_sources(tmp_path):
+    # an ncu summary gives `traffic` only while the source hash it records
+    # matches the kernel sources; otherwise (or with no summary) it is null
+    bench = _load_bench()
+    body = "# summary\n\n- kernel_source_sha: `%s`\n- dram_bytes_per_launch: 138362624\n"
+    current = tmp_path / "current.md"
+    current.write_text(body % bench.kernel_source_hash())
+    assert bench.profiled_traffic(str(current)) == 138362624.0
+    stale = tmp_path / "stale.md"
+    stale.write_text(body % "0000000000000000")
+    assert bench.profiled_traffic(str(stale)) is None
+    assert bench.profiled_traffic(str(tmp_path / "missing.md")) is None
