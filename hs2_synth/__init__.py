@@ -28,6 +28,8 @@ from .gen import (  # noqa: F401
     bf16_bits_to_f32,
     e4m3_value_table,
     fp8_quantise_pow2,
+    fp8_quantise_with_scales,
+    random_mantissa_scales,
     fp8_dequantise,
 )
 from .workloads import (  # noqa: F401

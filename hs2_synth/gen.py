@@ -124,6 +124,32 @@ def fp8_quantise_pow2(x: np.ndarray):
     return codes, scale.astype(np.float32)
 
 
+def fp8_quantise_with_scales(x: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """E4M3 codes of rows of x ([..., D]) for given fp32 per-row scales.
+
+    Each element is stored as the nearest E4M3 code of x / scale (computed in
+    float64 with the scale exactly as stored; ties to the even code; saturating
+    at 448), so the stored value is code * scale.  Returns uint8 codes [..., D].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    s = np.asarray(scale, dtype=np.float32).astype(np.float64)
+    return _nearest_e4m3(np.clip(x / s[..., None], -448.0, 448.0))
+
+
+def random_mantissa_scales(x: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """Per-row fp32 scales with an arbitrary (non-power-of-two) mantissa.
+
+    scale = max|x_row| / 448 * (1 + u_row / 2), rounded to fp32, with u_row a
+    uniform in [0, 1): every row fits the E4M3 range, and the scale's mantissa
+    bits are random, so a kernel that loses scale precision shows up in the
+    results (a power-of-two scale would hide it: its products are exact at any
+    precision).  Rows of zeros get 1.  Returns float32 [...].
+    """
+    amax = np.max(np.abs(np.asarray(x, dtype=np.float64)), axis=-1)
+    s = amax / 448.0 * (1.0 + 0.5 * np.asarray(u, dtype=np.float64).reshape(amax.shape))
+    return np.where(amax > 0, s, 1.0).astype(np.float32)
+
+
 def fp8_dequantise(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
     """Value of E4M3 codes times their row scale (float64); used to plant and check inputs."""
     c = np.asarray(codes, dtype=np.uint8)

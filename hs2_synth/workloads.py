@@ -26,6 +26,8 @@ from .gen import (
     f32_to_bf16_bits,
     bf16_bits_to_f32,
     fp8_quantise_pow2,
+    fp8_quantise_with_scales,
+    random_mantissa_scales,
 )
 
 
@@ -43,6 +45,9 @@ class AttnWorkload:
     seed: int
     topk: int = 1024
     window: int = 128
+    # E4M3 per-token scales: "pow2" (smallest power of two that fits the row)
+    # or "mantissa" (random non-power-of-two scales, see random_mantissa_scales)
+    fp8_scale: str = "pow2"
 
     @property
     def scale(self) -> float:
@@ -159,9 +164,16 @@ def make_attention_inputs(wl: AttnWorkload, needles: bool = True) -> AttnInputs:
     if wl.kv_dtype == "bf16":
         k, v = _bf16(kf), _bf16(vf)
         ks = vs = None
-    elif wl.kv_dtype == "fp8":
+    elif wl.kv_dtype == "fp8" and wl.fp8_scale == "pow2":
         k, ks = fp8_quantise_pow2(kf)
         v, vs = fp8_quantise_pow2(vf)
+    elif wl.kv_dtype == "fp8" and wl.fp8_scale == "mantissa":
+        n = wl.B * wl.L
+        ks = random_mantissa_scales(kf, uniform_stream(stream_seed(wl.seed, "k_scale"), n))
+        vs = random_mantissa_scales(vf, uniform_stream(stream_seed(wl.seed, "v_scale"), n))
+        ks, vs = ks.reshape(wl.B, wl.L), vs.reshape(wl.B, wl.L)
+        k = fp8_quantise_with_scales(kf, ks)
+        v = fp8_quantise_with_scales(vf, vs)
     else:
         raise ValueError(wl.kv_dtype)
     del kf, vf

@@ -73,16 +73,22 @@ def test_decode_bf16_32k():
     _check_block(WORKLOADS["decode_bf16_32k"])
 
 
-def test_decode_fp8_ragged():
-    _check_block(WORKLOADS["decode_fp8_256k"].resized(B=2, L=9007, n_needles=20))
+@pytest.mark.parametrize("fp8_scale", ["pow2", "mantissa"])
+def test_decode_fp8_ragged(fp8_scale):
+    # "mantissa": per-token scales with random mantissa bits, so the kernels'
+    # products with k_scale and v_scale are inexact at reduced precision
+    _check_block(WORKLOADS["decode_fp8_256k"].resized(B=2, L=9007, n_needles=20,
+                                                      fp8_scale=fp8_scale))
 
 
 def test_decode_fp8_256k():
     _check_block(WORKLOADS["decode_fp8_256k"])
 
 
-def test_chunk_fp8_small():
-    wl = WORKLOADS["chunk_fp8_1m"].resized(T=200, L=20011, n_needles=40, n_sparse=1)
+@pytest.mark.parametrize("fp8_scale", ["pow2", "mantissa"])
+def test_chunk_fp8_small(fp8_scale):
+    wl = WORKLOADS["chunk_fp8_1m"].resized(T=200, L=20011, n_needles=40, n_sparse=1,
+                                           fp8_scale=fp8_scale)
     rows = np.unique(np.r_[0, 199, np.random.default_rng(1).integers(0, 200, 30)])
     _check_block(wl, rows=rows)
 
@@ -174,13 +180,19 @@ def test_all_scores_tied_large_context():
 
 
 def test_chunk_fp8_1m_sampled_rows():
-    # the full 4096-query chunk over a 1M-token E4M3 cache, in the launch
-    # configuration of that shape; the oracle checks sampled query rows (first,
-    # middle, last, and rows that own planted needles) one by one
-    wl = WORKLOADS["chunk_fp8_1m"].resized(n_sparse=1)
+    # the full 4096-query chunk over a 1M-token E4M3 cache (per-token scales with
+    # random mantissas), in the launch configuration of that shape; the oracle
+    # checks 64 query rows one by one -- the first, the last, 8 rows that own
+    # planted needles, and the rest drawn from a seeded stream (they land in
+    # different 128-row groups and key splits) -- and all three sparse layers on
+    # those rows
+    wl = WORKLOADS["chunk_fp8_1m"].resized(fp8_scale="mantissa")
     inp = make_attention_inputs(wl)
-    needle_rows = sorted({int(t) for _, _, t in inp.needles})[:: max(1, len(inp.needles) // 3)][:3]
-    rows = np.unique(np.r_[0, 1, wl.T // 2, wl.T - 1, needle_rows])
+    rng = np.random.default_rng(2026)
+    needle_rows = sorted({int(t) for _, _, t in inp.needles})
+    rows = np.unique(np.r_[0, wl.T - 1, needle_rows[:: max(1, len(needle_rows) // 8)][:8]])
+    while rows.size < 64:
+        rows = np.unique(np.r_[rows, rng.integers(1, wl.T - 1, 64 - rows.size)])
     _check_block(wl, rows=rows, inp=inp)
 
 
