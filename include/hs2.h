@@ -176,15 +176,23 @@ HS2_API hs2_status hs2_sparse_attn(const void* Q, const hs2_kv_cache* kv, int B,
  * HS2_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU which loads libhs2 keeps
  * until the process exits.  It never calls cudaMalloc, cudaFree or any
  * allocating routine.
- *   - The first call on a device looks up that device's address of the array
- *     (cudaGetSymbolAddress, with the caller's current device); make that
- *     first call before any stream capture on the device.
- *   - A request whose workspace (hs2_full_attn_select_workspace) exceeds
- *     HS2_NOALLOC_SCRATCH_BYTES returns HS2_ERR_WORKSPACE and enqueues nothing.
- *     For example, 8 sequences of 32K positions need about 4.6 MB.
+ *   - Arguments are checked exactly as hs2_full_attn_select checks them
+ *     (HS2_ERR_INVALID_ARG / HS2_ERR_UNSUPPORTED) before the size: then a
+ *     request whose workspace (hs2_full_attn_select_workspace) exceeds
+ *     HS2_NOALLOC_SCRATCH_BYTES returns HS2_ERR_WORKSPACE.  Either way nothing
+ *     is enqueued.  For example, 8 sequences of 32K positions need 4.6 MB.
+ *   - The device address of the array is looked up (cudaGetSymbolAddress, on
+ *     the caller's current device) by every call made outside stream capture;
+ *     a call made while `stream` is being captured reuses the address found by
+ *     the last call on that device outside capture, so make one call on each
+ *     device before capturing it (the first call may also load the library's
+ *     kernels, which capture forbids).  After a cudaDeviceReset, call once
+ *     more outside capture before capturing again.
  *   - All calls on a device share the one array, and it keeps whatever the
- *     last call left there; the kernels clear the parts that must start at
- *     zero themselves.  Calls whose work overlaps on the GPU (different
+ *     last call left there.  Every call clears on `stream` the parts that must
+ *     start at zero: the fused kernel's arrival counters by a memset the call
+ *     enqueues before the kernel, the selection histograms inside the kernels
+ *     that fill them.  Calls whose work overlaps on the GPU (different
  *     streams, or different host threads) race on the array and must be
  *     serialised by the caller.
  * Outputs and status codes are those of hs2_full_attn_select.
@@ -223,6 +231,20 @@ HS2_API const char* hs2_status_string(hs2_status status);
  * enqueued by this call.
  */
 HS2_API hs2_status hs2_set_stage_events(void* begin_event, void* end_event);
+
+/*
+ * Fault injection, for testing failure detection without a GPU fault.  While
+ * extra_arrivals > 0, the group barriers of the fused full-attention kernel
+ * (head_dim 128, 32 query rows per group, several CTAs per group) wait for
+ * that many arrivals beyond the group's CTA count, which never come: every
+ * such wait gives up after wait_limit_ns nanoseconds (0 = the default, one
+ * second), raises HS2_ERR_TIMEOUT (read by hs2_last_device_status) and the
+ * kernel's CTAs return with their outputs unfinished.  wait_limit_ns also
+ * bounds those barriers when extra_arrivals is 0.  The setting applies to the
+ * full-attention calls made afterwards on this host thread; (0, 0) restores
+ * the defaults.  Nothing is enqueued by this call; it returns HS2_OK.
+ */
+HS2_API hs2_status hs2_set_fault_injection(unsigned extra_arrivals, unsigned long long wait_limit_ns);
 
 /* Library ABI version: 100 * major + minor. */
 HS2_API int hs2_version(void);

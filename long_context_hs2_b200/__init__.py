@@ -25,7 +25,8 @@ _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error",
 
 EXPORTED = ("hs2_bridge_kv", "hs2_full_attn_select_workspace", "hs2_full_attn_select",
             "hs2_full_attn_select_noalloc", "hs2_sparse_attn", "hs2_last_device_status",
-            "hs2_status_string", "hs2_version", "hs2_set_stage_events")
+            "hs2_status_string", "hs2_version", "hs2_set_stage_events",
+            "hs2_set_fault_injection")
 
 # Size of the scratch area built into the library for hs2_full_attn_select_noalloc.
 HS2_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -72,6 +73,8 @@ def load_library(path: str = LIB_PATH):
     lib.hs2_full_attn_select_noalloc.argtypes = [P, KV, i32, i32, i64, i32, i32, ctypes.c_float,
                                                  i32, i32, i32, P, P, P, P, P]
     lib.hs2_set_stage_events.restype = i32
+    lib.hs2_set_fault_injection.restype = i32
+    lib.hs2_set_fault_injection.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
     lib.hs2_set_stage_events.argtypes = [P, P]
     lib.hs2_sparse_attn.restype = i32
     lib.hs2_sparse_attn.argtypes = [P, KV, i32, i32, i64, i32, i32, ctypes.c_float, P, P, i32, i32,
@@ -172,3 +175,11 @@ def hs2_set_stage_events(begin=None, end=None):
             return e
         return e.cuda_event
     _check("hs2_set_stage_events", load_library().hs2_set_stage_events(handle(begin), handle(end)))
+
+
+def hs2_set_fault_injection(extra_arrivals: int = 0, wait_limit_ns: int = 0):
+    """Test hook: the fused kernel's group barriers wait for `extra_arrivals`
+    arrivals that never come and give up after `wait_limit_ns` (0: one second).
+    With no arguments, restores the defaults."""
+    _check("hs2_set_fault_injection",
+           load_library().hs2_set_fault_injection(int(extra_arrivals), int(wait_limit_ns)))

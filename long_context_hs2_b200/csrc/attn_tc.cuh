@@ -663,9 +663,14 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
 // Arrival at a group-wide barrier of CTAs through a global counter (zeroed
 // before the launch), then a bounded wait until `target` CTAs have arrived.
 // Whole CTA.  The CTAs of a group must be co-resident (cooperative launch).
-__device__ __forceinline__ void group_arrive_wait(unsigned* ctr, unsigned target) {
+// Returns false in every thread of the CTA when the wait gave up (after
+// limit_ns of %globaltimer, or 2^24 polls), having raised kStatusTimeout.
+__device__ __forceinline__ bool group_arrive_wait(unsigned* ctr, unsigned target,
+                                                  unsigned long long limit_ns) {
+  __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
+    int ok = 1;
     __threadfence();
     atomicAdd(ctr, 1u);
     const unsigned long long t0 = globaltimer();
@@ -673,15 +678,18 @@ __device__ __forceinline__ void group_arrive_wait(unsigned* ctr, unsigned target
       unsigned v;
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
       if (v >= target) break;
-      if (it >= (1u << 24) || ((it & 15u) == 15u && globaltimer() - t0 > kWaitLimitNs)) {
+      if (it >= (1u << 24) || ((it & 15u) == 15u && globaltimer() - t0 > limit_ns)) {
         raise_status(kStatusTimeout);
+        ok = 0;
         break;
       }
       __nanosleep(64);
     }
     __threadfence();
+    s_ok = ok;
   }
   __syncthreads();
+  return s_ok != 0;
 }
 
 // Fused decode pass: the partial pass of this CTA's (group, split), then --
@@ -753,8 +761,21 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   unsigned* gsync = p.grp_sync + 8 * grp;
+  const unsigned target = (unsigned)ns + p.barrier_extra;
+  // a group barrier that gave up ends the CTA: nothing is in flight (the
+  // partial pass has drained its TMA and MMA pipelines), so only the TMEM
+  // columns are released
+  auto give_up = [&]() {
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kTmemCols);
+    }
+  };
   tc_fence_before();
-  group_arrive_wait(gsync, (unsigned)ns);  // the group's partials are out
+  if (!group_arrive_wait(gsync, target, p.wait_limit_ns)) {  // the group's partials are out
+    give_up();
+    return;
+  }
   tc_fence_after();
 
   // --------------------------------------------------------- score pass
@@ -961,7 +982,10 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     auto list_g = [&](int q, int sp) {
       return p.sel_list + (row_of(q) * ns + sp) * (long long)p.split_keys;
     };
-    group_arrive_wait(gsync + 1, (unsigned)ns);  // level-1 counts complete
+    if (!group_arrive_wait(gsync + 1, target, p.wait_limit_ns)) {  // level-1 counts complete
+      give_up();
+      return;
+    }
 #pragma unroll 1
     for (int q = 0; q < G; ++q)
       if (active(q)) {
@@ -1005,7 +1029,11 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         }
         __syncthreads();  // s_res / s_w* are reused by the next row
       }
-    group_arrive_wait(gsync + 2, (unsigned)ns);  // every split's counts and b1 slice are out
+    // every split's counts and b1 slice are out
+    if (!group_arrive_wait(gsync + 2, target, p.wait_limit_ns)) {
+      give_up();
+      return;
+    }
 #pragma unroll 1
     for (int q = 0; q < G; ++q)
       if (active(q)) {

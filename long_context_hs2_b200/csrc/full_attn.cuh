@@ -49,6 +49,10 @@ struct FullAttnParams {
   int32_t* idx;                  // [B*T][slots]
   int32_t* n_sel;                // [B*T]
   int topk, slots, fuse_select;
+  // the group barriers' wait limit, and arrivals they wait for beyond the
+  // group's CTA count (non-zero only under fault injection)
+  unsigned long long wait_limit_ns;
+  unsigned barrier_extra;
 };
 
 template <int D, bool FP8>

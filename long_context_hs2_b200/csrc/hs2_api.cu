@@ -72,6 +72,11 @@ int sm_count() {
 // ------------------------------------------- optional stage timing --
 thread_local cudaEvent_t t_stage_begin = nullptr, t_stage_end = nullptr;
 
+// ------------------------------------------------- fault injection --
+constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;
+thread_local unsigned t_barrier_extra = 0;
+thread_local unsigned long long t_wait_limit_ns = kDefaultWaitLimitNs;
+
 // Records the caller's stage event (if any) on s; an external event node when
 // s is being captured into a graph.
 cudaError_t stage_mark(cudaStream_t s, bool begin) {
@@ -101,6 +106,26 @@ bool check_attn_shape(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt) {
   if (!(D == 64 || D == 128)) return false;
   if (dt != HS2_KV_BF16 && dt != HS2_KV_FP8_E4M3) return false;
   return true;
+}
+
+// Host-side checks of hs2_full_attn_select's arguments, before any workspace
+// or device state is looked at.
+hs2_status check_full_args(const void* Q, const hs2_kv_cache* kv, int B, int T, int64_t L, int H,
+                           int D, float scale, int topk, int window, hs2_kv_dtype dt,
+                           const float* O, const float* lse, const int32_t* idx,
+                           const int32_t* n_sel) {
+  if (!Q || !kv || !kv->k || !kv->v || !O || !idx || !n_sel) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(kv->k) || !aligned16(kv->v) || !aligned16(O) ||
+      !aligned4(idx) || !aligned4(n_sel) || (lse && !aligned4(lse)))
+    return HS2_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || L < T || topk < 0 || window < 1 || !std::isfinite(scale))
+    return HS2_ERR_INVALID_ARG;
+  if (dt == HS2_KV_FP8_E4M3 && (!kv->k_scale || !kv->v_scale || !aligned4(kv->k_scale) ||
+                                !aligned4(kv->v_scale)))
+    return HS2_ERR_INVALID_ARG;
+  if (!check_attn_shape(B, T, L, H, D, dt) || topk + window > 4096) return HS2_ERR_UNSUPPORTED;
+  if (dt == HS2_KV_FP8_E4M3 && D != 128) return HS2_ERR_UNSUPPORTED;
+  return HS2_OK;
 }
 
 bool make_full_plan(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt, FullPlan* pl) {
@@ -313,6 +338,12 @@ extern "C" {
 
 int hs2_version(void) { return 101; }
 
+hs2_status hs2_set_fault_injection(unsigned extra_arrivals, unsigned long long wait_limit_ns) {
+  t_barrier_extra = extra_arrivals;
+  t_wait_limit_ns = wait_limit_ns ? wait_limit_ns : kDefaultWaitLimitNs;
+  return HS2_OK;
+}
+
 hs2_status hs2_set_stage_events(void* begin_event, void* end_event) {
   if ((begin_event == nullptr) != (end_event == nullptr)) return HS2_ERR_INVALID_ARG;
   t_stage_begin = static_cast<cudaEvent_t>(begin_event);
@@ -357,17 +388,9 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
                                 hs2_kv_dtype dt, float* O, float* lse, int32_t* idx,
                                 int32_t* n_sel, void* workspace, size_t workspace_bytes,
                                 hs2_stream_t stream) {
-  if (!Q || !kv || !kv->k || !kv->v || !O || !idx || !n_sel) return HS2_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(kv->k) || !aligned16(kv->v) || !aligned16(O) ||
-      !aligned4(idx) || !aligned4(n_sel) || (lse && !aligned4(lse)))
-    return HS2_ERR_INVALID_ARG;
-  if (B < 1 || T < 1 || L < T || topk < 0 || window < 1 || !std::isfinite(scale))
-    return HS2_ERR_INVALID_ARG;
-  if (dt == HS2_KV_FP8_E4M3 && (!kv->k_scale || !kv->v_scale || !aligned4(kv->k_scale) ||
-                                !aligned4(kv->v_scale)))
-    return HS2_ERR_INVALID_ARG;
-  if (!check_attn_shape(B, T, L, H, D, dt) || topk + window > 4096) return HS2_ERR_UNSUPPORTED;
-  if (dt == HS2_KV_FP8_E4M3 && D != 128) return HS2_ERR_UNSUPPORTED;
+  const hs2_status chk = check_full_args(Q, kv, B, T, L, H, D, scale, topk, window, dt, O, lse,
+                                         idx, n_sel);
+  if (chk != HS2_OK) return chk;
   FullPlan pl;
   make_full_plan(B, T, L, H, D, dt, &pl);
   if (!workspace || workspace_bytes < pl.total || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
@@ -426,6 +449,8 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
   fp.topk = topk;
   fp.slots = topk + window;
   fp.fuse_select = 0;
+  fp.wait_limit_ns = t_wait_limit_ns;
+  fp.barrier_extra = t_barrier_extra;
 
   cudaStream_t s = (cudaStream_t)stream;
   if (pl.fused)
@@ -487,6 +512,26 @@ hs2_status hs2_sparse_attn(const void* Q, const hs2_kv_cache* kv, int B, int T, 
 
 }  // extern "C"
 
+namespace {
+
+void fill_bridge_params(BridgeParams* p, const hs2_kv_cache* caches, int n_layers, bool fp8,
+                        int64_t T, int64_t row_offset, int hidden) {
+  std::memset(p, 0, sizeof(*p));
+  for (int l = 0; l < n_layers; ++l) {
+    p->k[l] = caches[l].k;
+    p->v[l] = caches[l].v;
+    p->k_scale[l] = fp8 ? caches[l].k_scale : nullptr;
+    p->v_scale[l] = fp8 ? caches[l].v_scale : nullptr;
+  }
+  p->T = T;
+  p->row_offset = row_offset;
+  p->hidden = hidden;
+  p->n_layers = n_layers;
+  p->fp8 = fp8 ? 1 : 0;
+}
+
+}  // namespace
+
 extern "C" hs2_status hs2_bridge_kv(const void* X, int64_t T, int hidden, const void* Wt,
                                     int n_layers, int D, hs2_kv_dtype out_dtype,
                                     const hs2_kv_cache* caches, int64_t cache_row_offset,
@@ -509,18 +554,7 @@ extern "C" hs2_status hs2_bridge_kv(const void* X, int64_t T, int hidden, const 
       !make_map_2d(&wm, Wt, (uint64_t)n_layers * kBrBN, (uint64_t)hidden, 2, kBrBK, kBrBN))
     return HS2_ERR_CUDA;
   BridgeParams p;
-  std::memset(&p, 0, sizeof(p));
-  for (int l = 0; l < n_layers; ++l) {
-    p.k[l] = caches[l].k;
-    p.v[l] = caches[l].v;
-    p.k_scale[l] = fp8 ? caches[l].k_scale : nullptr;
-    p.v_scale[l] = fp8 ? caches[l].v_scale : nullptr;
-  }
-  p.T = T;
-  p.row_offset = cache_row_offset;
-  p.hidden = hidden;
-  p.n_layers = n_layers;
-  p.fp8 = fp8 ? 1 : 0;
+  fill_bridge_params(&p, caches, n_layers, fp8, T, cache_row_offset, hidden);
   if (!set_smem(bridge_gemm_kernel, kBrSmemBytes)) return HS2_ERR_CUDA;
   const long long tiles = (T + kBrBM - 1) / kBrBM * n_layers;
   const int grid = (int)std::min<long long>(tiles, sm_count());
@@ -540,15 +574,23 @@ constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
 
-// Device address of the scratch array on the current device, looked up once
-// per device (the host-side name of the array is only a stand-in: a kernel
-// handed it would fault or read the wrong memory).
-hs2_status noalloc_scratch(void** out) {
+// Device address of the scratch array on the current device.  Outside stream
+// capture it is looked up on every call (a device reset reloads the module,
+// and the array may then sit elsewhere); under capture the address of the last
+// lookup on this device is used, since a lookup may load the module, which
+// capture forbids.  (The host-side name of the array is only a stand-in: a
+// kernel handed it would fault or read the wrong memory.)
+hs2_status noalloc_scratch(cudaStream_t s, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return HS2_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return HS2_ERR_UNSUPPORTED;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return HS2_ERR_CUDA;
+  }
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (cs == cudaStreamCaptureStatusNone || !g_scratch_ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
       cudaGetLastError();
@@ -567,13 +609,16 @@ extern "C" hs2_status hs2_full_attn_select_noalloc(const void* Q, const hs2_kv_c
                                                    int topk, int window, hs2_kv_dtype dt,
                                                    float* O, float* lse, int32_t* idx,
                                                    int32_t* n_sel, hs2_stream_t stream) {
+  // arguments first, exactly as hs2_full_attn_select checks them; then the size
+  const hs2_status chk = check_full_args(Q, kv, B, T, L, H, D, scale, topk, window, dt, O, lse,
+                                         idx, n_sel);
+  if (chk != HS2_OK) return chk;
   const size_t need = hs2_full_attn_select_workspace(B, T, L, H, D, topk, window, dt);
+  if (need == 0) return HS2_ERR_UNSUPPORTED;
   if (need > HS2_NOALLOC_SCRATCH_BYTES) return HS2_ERR_WORKSPACE;
   void* scratch = nullptr;
-  if (need > 0) {  // need == 0: invalid shape, reported by the call below
-    const hs2_status st = noalloc_scratch(&scratch);
-    if (st != HS2_OK) return st;
-  }
+  const hs2_status st = noalloc_scratch((cudaStream_t)stream, &scratch);
+  if (st != HS2_OK) return st;
   return hs2_full_attn_select(Q, kv, B, T, L, H, D, scale, topk, window, dt, O, lse, idx, n_sel,
-                              scratch, need > 0 ? (size_t)HS2_NOALLOC_SCRATCH_BYTES : 0, stream);
+                              scratch, (size_t)HS2_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -92,6 +92,22 @@ def test_sparse_attn_rejects_bad_arguments(lib):
     assert f(16, ctypes.byref(kv8), 1, 1, 64, 32, 64, 0.1, 16, 16, 8, 1, 16, None) == 2  # fp8 needs D=128
 
 
+def test_noalloc_checks_arguments_before_the_size(lib):
+    # a request far beyond the built-in scratch, but with a null or misaligned
+    # pointer: the argument error is reported first, and nothing is enqueued
+    kv = hs2.hs2_kv_cache(16, 16, None, None)
+    f = lib.hs2_full_attn_select_noalloc
+    B, T, L, H, D = 64, 1, 65536, 32, 128
+    assert f(None, ctypes.byref(kv), B, T, L, H, D, 0.1, 1024, 128, 0, 16, None, 16, 16, None) == 1
+    assert f(16, ctypes.byref(kv), B, T, L, H, D, 0.1, 1024, 128, 0, 8, None, 16, 16, None) == 1
+    assert f(16, ctypes.byref(kv), B, T, L, H, 96, 0.1, 1024, 128, 0, 16, None, 16, 16, None) == 2
+
+
+def test_fault_injection_setter(lib):
+    assert lib.hs2_set_fault_injection(1, 2000000) == 0
+    assert lib.hs2_set_fault_injection(0, 0) == 0
+
+
 def test_stage_events_pairing(lib):
     assert lib.hs2_set_stage_events(ctypes.c_void_p(16), None) == 1
     assert lib.hs2_set_stage_events(None, ctypes.c_void_p(16)) == 1
