@@ -175,6 +175,14 @@ def oracle_rows_per_s(inp, rows, n_sparse):
     return len(rows) / dt, dt, oracle.threads()
 
 
+def bench_config(wl, world):
+    """The `config` object of both arms' JSON lines (the same keys and values)."""
+    return {"workload": WORKLOAD, "B": wl.B, "T": wl.T, "L": wl.L, "H": wl.H, "D": wl.D,
+            "kv": wl.kv_dtype, "topk": wl.topk, "window": wl.window,
+            "sparse_layers": wl.n_sparse, "parallelism": "replicas (dp%d)" % world,
+            "l2": "flushed before each step (512 MB write, then read back)"}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
@@ -189,16 +197,14 @@ def run_reference(args, world, rank):
         rows = np.array([s % (wl.B * wl.T)])
         _, dt, cores = oracle_rows_per_s(inp, rows, wl.n_sparse)
         times.append(dt)
-    ms = 1000.0 * sum(times) / len(times)
+    ms = 1000.0 * statistics.median(times)
     value = 1000.0 / ms
     line = {
         "impl": "reference", "metric": "hybrid-block decode tokens/s", "value": value,
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": wl.B, "T": wl.T, "L": wl.L, "H": wl.H, "D": wl.D,
-                   "kv": wl.kv_dtype, "topk": wl.topk, "window": wl.window,
-                   "sparse_layers": wl.n_sparse},
+        "config": bench_config(wl, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": "1 of the 8 sequences per step (full attention + selection "
                                    "+ 3 sparse layers), plain C++ fp64 oracle"},
@@ -324,10 +330,11 @@ def bench_other_configs(torch, hs2, stream, flush_fn, peak_gbs, peak_tflops):
             entry.update({"full_gbs": full_bytes / (res["full"] * 1e-3) / 1e9,
                           "full_frac_hbm": full_bytes / (res["full"] * 1e-3) / 1e9 / peak_gbs})
         else:
-            # causal (query, key, head) triples; QK^T + PV, and the score pass's QK^T again
+            # the method's work: QK^T and PV over the causal (query, key, head)
+            # triples (a recomputation of QK^T for the scores is not counted)
             triples = sum((L - T + t + 1) for t in range(T)) * H
-            flops = triples * 4 * D + triples * 2 * D
-            exps = 2 * triples
+            flops = triples * 4 * D
+            exps = triples
             entry.update({"full_tflops": flops / (res["full"] * 1e-3) / 1e12,
                           "full_frac_tensor": flops / (res["full"] * 1e-3) / 1e12 / peak_tflops,
                           "full_exp_per_s": exps / (res["full"] * 1e-3)})
@@ -339,7 +346,10 @@ def bench_other_configs(torch, hs2, stream, flush_fn, peak_gbs, peak_tflops):
 
 # ------------------------------------------------------------------ GPU arm --
 PARTIAL_PROFILE = os.path.join(ROOT, "profiles", "attn_tc_fused_decode_bf16_32k.md")
-KERNEL_SOURCES = ("attn_tc.cuh", "tc_common.cuh", "hs2_common.cuh", "full_attn.cuh", "select.cuh")
+# the fused kernel's sources and the host code that plans its launch (splits,
+# keys per split, fused selection, retained logits)
+KERNEL_SOURCES = ("attn_tc.cuh", "tc_common.cuh", "hs2_common.cuh", "full_attn.cuh", "select.cuh",
+                  "hs2_api.cu")
 
 
 def kernel_source_hash():
@@ -536,7 +546,7 @@ def run_hs2(args, world, rank, local):
     e2e_ms = [a.elapsed_time(c) for a, c in e2e_ev]
 
     def agg(xs):
-        return max_over_ranks(float(np.mean(xs)), world, "cuda")
+        return max_over_ranks(float(np.median(xs)), world, "cuda")
 
     ms = agg(step_ms)
     full = agg(full_ms)
@@ -582,10 +592,7 @@ def run_hs2(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": B, "T": T, "L": L, "H": H, "D": D,
-                   "kv": "bf16", "topk": wl.topk, "window": wl.window,
-                   "sparse_layers": wl.n_sparse, "parallelism": "replicas (dp%d)" % world,
-                   "l2": "flushed before each step (512 MB write, then read back)"},
+        "config": bench_config(WORKLOADS[WORKLOAD], world),
         "e2e": {"value": job_throughput(B * T, world, e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
