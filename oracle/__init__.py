@@ -60,6 +60,8 @@ def _configure(lib):
                                           i32, i32, P, i64, P, P, P, P, P]
     lib.hs2o_select.restype = i32
     lib.hs2o_select.argtypes = [P, i64, i32, i32, P, P]
+    lib.hs2o_select_blocks.restype = i32
+    lib.hs2o_select_blocks.argtypes = [P, i64, i32, i32, i32, P, P]
     lib.hs2o_sparse_attn.restype = i32
     lib.hs2o_sparse_attn.argtypes = [P, i32, P, P, P, P, i32, i32, i64, i32, i32, dbl,
                                      P, P, i32, P, i64, P]
@@ -204,6 +206,20 @@ def select(score_row: np.ndarray, i: int, topk: int, window: int):
     ns = np.zeros(1, dtype=np.int32)
     if lib.hs2o_select(_p(s), int(i), topk, window, _p(idx), _p(ns)) != 0:
         raise ValueError("hs2o_select: invalid arguments")
+    return idx, int(ns[0])
+
+
+def select_blocks(score_row: np.ndarray, i: int, topk: int, window: int, block: int = 64):
+    """Block-level selection of query position i from a head-summed score row
+    score[0..i] (dpshk.com explainer, section 03: the earlier HySparse chose
+    history in blocks of 64 tokens): the topk/block candidate blocks of largest
+    summed score, ties to the lower block, plus the window."""
+    lib = _load()
+    s = _c(score_row, np.float64)
+    idx = np.zeros(topk + window, dtype=np.int32)
+    ns = np.zeros(1, dtype=np.int32)
+    if lib.hs2o_select_blocks(_p(s), int(i), topk, window, block, _p(idx), _p(ns)) != 0:
+        raise ValueError("hs2o_select_blocks: invalid arguments")
     return idx, int(ns[0])
 
 

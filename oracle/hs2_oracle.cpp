@@ -169,6 +169,44 @@ void select_row(const double* score, int64_t i, int topk, int window, int32_t* i
   *n_sel_out = (int32_t)sel.size();
 }
 
+// Block-level selection, the granularity of the HySparse generation before
+// HySparse2 (dpshk.com explainer, section 03: history chosen in blocks of 64
+// tokens, so one useful token takes a whole block of the budget; cnyes.com
+// article, section "檢索精確到token": the ablation keeps the same budget and
+// compares block-level with token-level choice).  Readings where the pages are
+// silent: the candidate positions are the token-level ones, C = {0 .. i-window};
+// block b holds positions b*block .. b*block+block-1 and is a candidate when it
+// holds a candidate position; its score is the sum of the head-summed scores of
+// its candidate positions; blocks are ordered by (score descending, block index
+// ascending) and the first min(topk / block, #candidate blocks) are selected;
+// S = the candidate positions of the selected blocks, union the window, in
+// ascending order, padded with -1 to topk + window slots.
+void select_blocks_row(const double* score, int64_t i, int topk, int window, int block,
+                       int32_t* idx_out, int32_t* n_sel_out) {
+  const int64_t last = i - window;  // last candidate position (none when < 0)
+  const int64_t nblk = last < 0 ? 0 : last / block + 1;
+  std::vector<double> bsum((size_t)nblk, 0.0);
+  for (int64_t j = 0; j <= last; ++j) bsum[(size_t)(j / block)] += score[j];
+  std::vector<int64_t> order((size_t)nblk);
+  for (int64_t b = 0; b < nblk; ++b) order[(size_t)b] = b;
+  std::sort(order.begin(), order.end(), [&](int64_t a, int64_t b) {
+    if (bsum[(size_t)a] != bsum[(size_t)b]) return bsum[(size_t)a] > bsum[(size_t)b];
+    return b > a;  // equal sums: the lower block first
+  });
+  const int64_t keep = std::min<int64_t>(topk / block, nblk);
+  std::vector<int64_t> sel;
+  for (int64_t n = 0; n < keep; ++n) {
+    const int64_t b = order[(size_t)n];
+    for (int64_t j = b * block; j < std::min<int64_t>((b + 1) * block, last + 1); ++j)
+      sel.push_back(j);
+  }
+  for (int64_t w = std::max<int64_t>(0, i - window + 1); w <= i; ++w) sel.push_back(w);
+  std::sort(sel.begin(), sel.end());
+  const int slots = topk + window;
+  for (int n = 0; n < slots; ++n) idx_out[n] = n < (int)sel.size() ? (int32_t)sel[n] : -1;
+  *n_sel_out = (int32_t)sel.size();
+}
+
 constexpr int64_t kChunk = 2048;  // fixed work-item size: keeps sums independent of threads
 
 }  // namespace
@@ -327,6 +365,17 @@ int hs2o_select(const double* score, int64_t i, int topk, int window, int32_t* i
                 int32_t* n_sel) {
   if (!score || !idx || !n_sel || i < 0 || topk < 0 || window < 1) return 1;
   select_row(score, i, topk, window, idx, n_sel);
+  return 0;
+}
+
+// Block-level selection alone, from a caller-supplied score row score[0..i]
+// (select_blocks_row above).  topk must be a multiple of block.
+int hs2o_select_blocks(const double* score, int64_t i, int topk, int window, int block,
+                       int32_t* idx, int32_t* n_sel) {
+  if (!score || !idx || !n_sel || i < 0 || topk < 0 || window < 1 || block < 1 ||
+      topk % block != 0)
+    return 1;
+  select_blocks_row(score, i, topk, window, block, idx, n_sel);
   return 0;
 }
 

@@ -250,6 +250,57 @@ def check_all_equal_keys():
     assert np.array_equal(r["idx"][0], expect)
 
 
+# -------------------------------------------------- block-level selection --
+def check_select_blocks_of_one_are_token_level():
+    # blocks of a single position are the token-level selection (pinned above
+    # against numpy's lexsort; compared with it directly here)
+    rng = np.random.default_rng(51)
+    for trial in range(40):
+        n = int(rng.integers(1, 300))
+        score = rng.integers(0, 5, n).astype(np.float64) if trial % 2 else rng.random(n)
+        topk, window = int(rng.integers(0, 40)), int(rng.integers(1, 20))
+        idx, ns = oracle.select_blocks(score, n - 1, topk, window, block=1)
+        ref = _lexsort_select(score, n - 1, topk, window)
+        assert ns == len(ref) and np.array_equal(idx[:ns], ref)
+
+
+def check_select_blocks_bruteforce_rank():
+    # a block is kept iff fewer than topk/block candidate blocks outrank it
+    # (larger summed score, or equal and lower index): pairwise counts, no sort
+    rng = np.random.default_rng(52)
+    for trial in range(60):
+        n = int(rng.integers(1, 400))
+        block = int(rng.choice([2, 3, 4, 8, 64]))
+        score = rng.integers(0, 3, n).astype(np.float64) if trial % 3 == 0 else rng.random(n)
+        window = int(rng.integers(1, 30))
+        kb = int(rng.integers(0, 12))
+        i = n - 1
+        idx, ns = oracle.select_blocks(score, i, kb * block, window, block=block)
+        last = i - window
+        sums = {}
+        for j in range(0, last + 1):
+            sums[j // block] = sums.get(j // block, 0.0) + score[j]
+        chosen = set()
+        for b, sb in sums.items():
+            rank = sum(1 for c, sc in sums.items() if sc > sb or (sc == sb and c < b))
+            if rank < kb:
+                chosen |= {j for j in range(b * block, (b + 1) * block) if j <= last}
+        chosen |= set(range(max(0, i - window + 1), i + 1))
+        assert ns == len(chosen)
+        assert idx[:ns].tolist() == sorted(chosen) and (idx[ns:] == -1).all()
+
+
+def check_golden_worked_block_selection():
+    with open(os.path.join(GOLDEN, "worked_block_selection.json")) as f:
+        g = json.load(f)
+    score = np.array(g["score"], dtype=np.float64)
+    for case in g["cases"]:
+        idx, ns = oracle.select_blocks(score, g["i"], case["topk"], g["window"], g["block"])
+        assert idx[:ns].tolist() == case["selected"]
+    idx, ns = oracle.select(score, g["i"], 4, g["window"])
+    assert idx[:ns].tolist() == g["token_level_topk4"]
+
+
 # ------------------------------------------------------------ sparse layer --
 def check_sparse_equals_dense():
     rng = np.random.default_rng(41)
@@ -302,5 +353,6 @@ ALL_CHECKS = [
     check_bridge_numpy, check_bridge_identity, check_attention_vs_torch,
     check_scores_sum_to_heads, check_select_vs_lexsort, check_select_bruteforce_rank,
     check_all_equal_keys, check_sparse_equals_dense, check_sparse_vs_torch,
-    check_golden_worked_example,
+    check_golden_worked_example, check_select_blocks_of_one_are_token_level,
+    check_select_blocks_bruteforce_rank, check_golden_worked_block_selection,
 ]

@@ -44,6 +44,14 @@ MUTANTS = {
                                  "for (int d = 0; d < D; ++d) acc[h * D + d] += p[(size_t)((h + 1) % H) * n + j] * vj[d];"),
     "fp8_value_scale_ignored": ("if (fp8) return e4m3_to_f64(((const uint8_t*)base)[off]) * (double)sc[(int64_t)b * L + j];",
                                 "if (fp8) return e4m3_to_f64(((const uint8_t*)base)[off]) * (double)sc[(int64_t)b * L];"),
+    "block_score_is_max_not_sum": ("for (int64_t j = 0; j <= last; ++j) bsum[(size_t)(j / block)] += score[j];",
+                                   "for (int64_t j = 0; j <= last; ++j) bsum[(size_t)(j / block)] = std::max(bsum[(size_t)(j / block)], score[j]);"),
+    "partial_boundary_block_not_counted": ("const int64_t keep = std::min<int64_t>(topk / block, nblk);",
+                                           "const int64_t keep = std::min<int64_t>(topk / block, (last + 1) / block);"),
+    "block_ties_to_higher_block": ("return b > a;  // equal sums: the lower block first",
+                                   "return a > b;  // equal sums: the lower block first"),
+    "boundary_block_overlaps_window": ("for (int64_t j = b * block; j < std::min<int64_t>((b + 1) * block, last + 1); ++j)",
+                                       "for (int64_t j = b * block; j < (b + 1) * block; ++j)"),
 }
 
 
