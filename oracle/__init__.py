@@ -60,6 +60,9 @@ def _configure(lib):
                                           i32, i32, P, i64, P, P, P, P, P]
     lib.hs2o_select.restype = i32
     lib.hs2o_select.argtypes = [P, i64, i32, i32, P, P]
+    lib.hs2o_attn_slice.restype = i32
+    lib.hs2o_attn_slice.argtypes = [P, i32, P, P, P, P, i32, i32, i64, i64, i32, i32, dbl, i32, P,
+                                    P, i64, P, P, P]
     lib.hs2o_select_blocks.restype = i32
     lib.hs2o_select_blocks.argtypes = [P, i64, i32, i32, i32, P, P]
     lib.hs2o_sparse_attn.restype = i32
@@ -193,6 +196,44 @@ def full_attn_select(q, k, v, k_scale=None, v_scale=None, *, scale: float, topk:
     if rc != 0:
         raise ValueError("hs2o_full_attn_select: invalid arguments")
     out = dict(o=o, lse=lse, idx=idx, n_sel=nsel)
+    if want_score:
+        out["score"] = sc
+    return out
+
+
+def attn_slice(q, k, v, k_scale=None, v_scale=None, *, qpos: int, scale: float, window: int = 128,
+               lse_in=None, rows=None, want_score: bool = False):
+    """Attention of the queries over one slice of a context split across devices
+    (dpshk.com explainer, section 05: million-token contexts): the slice's own
+    normaliser lse and output O (normalised over the slice), and, if asked, the
+    head-summed scores of the slice's candidates under lse_in (the normaliser
+    over the whole context; the slice's own when None).
+
+    q: uint16 [B, T, H, D]; k, v: the slice [B, L_slice, D]; query t sits at
+    slice-relative position qpos + t.  lse_in: [B*T, H] float64 or None.
+    Returns dict with o [n, H, D], lse [n, H] and optionally score [n, L_slice].
+    """
+    lib = _load()
+    q = _c(q, np.uint16)
+    fp8 = k.dtype == np.uint8
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    ks = _c(k_scale, np.float32)
+    vs = _c(v_scale, np.float32)
+    B, T, H, D = q.shape
+    L = k.shape[1]
+    rows_a = None if rows is None else _c(rows, np.int64)
+    n = B * T if rows_a is None else len(rows_a)
+    li = None if lse_in is None else _c(lse_in, np.float64)
+    o = np.zeros((n, H, D))
+    lse = np.zeros((n, H))
+    sc = np.zeros((n, L)) if want_score else None
+    rc = lib.hs2o_attn_slice(_p(q), int(fp8), _p(k), _p(v), _p(ks), _p(vs), B, T, L, int(qpos), H,
+                             D, float(scale), int(window), _p(li), _p(rows_a), n, _p(o), _p(lse),
+                             _p(sc))
+    if rc != 0:
+        raise ValueError("hs2o_attn_slice: invalid arguments")
+    out = dict(o=o, lse=lse)
     if want_score:
         out["score"] = sc
     return out

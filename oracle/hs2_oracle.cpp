@@ -360,6 +360,77 @@ int hs2o_full_attn_select(const uint16_t* Q, int kv_fp8, const void* K, const vo
   return 0;
 }
 
+// One slice of a context held across several devices (context parallelism of
+// the full-attention layer; the pages analyse contexts of a million tokens:
+// dpshk.com explainer, section 05).  The slice holds L_slice consecutive
+// positions of each sequence; query t sits at slice-relative position
+// i = qpos + t (it may lie beyond the slice, or before it).  For each listed
+// row (b, t) and head h, over the slice's keys j with 0 <= j < L_slice, j <= i:
+//   s_hj = scale * <q_h, k_j>,  lse_h = log sum_j exp(s_hj)  (-inf if no key)
+//   O_h  = sum_j exp(s_hj - lse_h) v_j                       (0 if no key)
+//   score_j = sum_h exp(s_hj - lse_ref_h) for the slice's candidates
+//             j <= i - window, where lse_ref = lse_in (the normaliser over the
+//             whole context) when given, else the slice's own lse.
+// Layouts as hs2o_full_attn_select: O [n_rows][H][D], lse [n_rows][H],
+// score [n_rows][L_slice] (0 for non-candidates); lse_in [B*T][H].  With the
+// slice = the whole cache (qpos = L - T) this is hs2o_full_attn_select's
+// attention and score.
+int hs2o_attn_slice(const uint16_t* Q, int kv_fp8, const void* K, const void* V,
+                    const float* k_scale, const float* v_scale, int B, int T, int64_t L_slice,
+                    int64_t qpos, int H, int D, double scale, int window, const double* lse_in,
+                    const int64_t* rows, int64_t n_rows, double* O, double* lse, double* score) {
+  if (!Q || !K || !V || B < 1 || T < 1 || L_slice < 1 || H < 1 || D < 1 || window < 1) return 1;
+  if (kv_fp8 && (!k_scale || !v_scale)) return 1;
+  if (!rows) n_rows = (int64_t)B * T;
+  const Cache kv{kv_fp8, K, V, k_scale, v_scale, L_slice, D};
+  parallel_for(n_rows, n_threads(), [&](int64_t r) {
+    const int64_t bt = rows ? rows[r] : r;
+    const int b = (int)(bt / T), t = (int)(bt % T);
+    const int64_t i = qpos + t;
+    const int64_t n = std::max<int64_t>(0, std::min<int64_t>(L_slice, i + 1));  // visible keys
+    std::vector<double> s((size_t)H * std::max<int64_t>(n, 1));
+    for (int64_t j = 0; j < n; ++j)
+      for (int h = 0; h < H; ++h) {
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d)
+          acc += bf16_to_f64(Q[((int64_t)bt * H + h) * D + d]) * kv.key(b, j, d);
+        s[(size_t)h * n + j] = scale * acc;
+      }
+    std::vector<double> lse_row(H, -INFINITY);
+    for (int h = 0; h < H; ++h) {
+      if (n == 0) continue;
+      double m = -INFINITY;
+      for (int64_t j = 0; j < n; ++j) m = std::max(m, s[(size_t)h * n + j]);
+      double l = 0.0;
+      for (int64_t j = 0; j < n; ++j) l += std::exp(s[(size_t)h * n + j] - m);
+      lse_row[h] = std::log(l) + m;
+    }
+    if (lse)
+      for (int h = 0; h < H; ++h) lse[(size_t)r * H + h] = lse_row[h];
+    if (O)
+      for (int h = 0; h < H; ++h)
+        for (int d = 0; d < D; ++d) {
+          double o = 0.0;
+          for (int64_t j = 0; j < n; ++j)
+            o += std::exp(s[(size_t)h * n + j] - lse_row[h]) * kv.val(b, j, d);
+          O[((size_t)r * H + h) * D + d] = o;
+        }
+    if (score) {
+      double* srow = score + (size_t)r * L_slice;
+      for (int64_t j = 0; j < L_slice; ++j) srow[j] = 0.0;
+      for (int64_t j = 0; j < n && j <= i - window; ++j) {
+        double acc = 0.0;
+        for (int h = 0; h < H; ++h) {
+          const double ref = lse_in ? lse_in[(size_t)bt * H + h] : lse_row[h];
+          acc += std::exp(s[(size_t)h * n + j] - ref);
+        }
+        srow[j] = acc;
+      }
+    }
+  });
+  return 0;
+}
+
 // Selection alone, from a caller-supplied score row score[0..i].
 int hs2o_select(const double* score, int64_t i, int topk, int window, int32_t* idx,
                 int32_t* n_sel) {

@@ -250,6 +250,48 @@ def check_all_equal_keys():
     assert np.array_equal(r["idx"][0], expect)
 
 
+# ------------------------------------------- context-parallel slice --
+def check_slice_of_the_whole_cache_is_full_attention():
+    rng = np.random.default_rng(61)
+    for fp8 in (False, True):
+        B, T, H, D, L = 2, 6, 4, 16, 260
+        q, k, v, ks, vs, *_ = _small_attn(rng, B, T, L, H, D, fp8)
+        r = oracle.full_attn_select(q, k, v, ks, vs, scale=0.3, topk=16, window=8, want_score=True)
+        sl = oracle.attn_slice(q, k, v, ks, vs, qpos=L - T, scale=0.3, window=8, want_score=True)
+        assert np.allclose(sl["o"], r["o"], rtol=1e-12, atol=1e-14)
+        assert np.allclose(sl["lse"], r["lse"], rtol=1e-13, atol=1e-13)
+        cand = np.arange(L)[None, :] <= (L - T + np.tile(np.arange(T), B))[:, None] - 8
+        assert np.allclose(sl["score"], np.where(cand, r["score"], 0.0), rtol=1e-11, atol=1e-15)
+
+
+def check_slice_vs_torch():
+    # slices that lie before, around and after the queries, with a given
+    # normaliser for the scores
+    rng = np.random.default_rng(62)
+    B, T, H, D, Ls, window = 1, 5, 3, 8, 40, 4
+    q, k, v, ks, vs, qf, kf, vf = _small_attn(rng, B, T, Ls, H, D, False)
+    lse_in = rng.normal(3.0, 1.0, (B * T, H))
+    for qpos in (100, 38, 20, 2, -3):
+        sl = oracle.attn_slice(q, k, v, qpos=qpos, scale=0.4, window=window, lse_in=lse_in,
+                               want_score=True)
+        s = torch.einsum("thd,ld->thl", torch.from_numpy(qf[0]), torch.from_numpy(kf[0])) * 0.4
+        pos = torch.arange(Ls)
+        i = qpos + torch.arange(T)
+        vis = pos[None, :] <= i[:, None]                                    # [T, Ls]
+        sm = s.masked_fill(~vis[:, None, :], float("-inf"))
+        lse = torch.logsumexp(sm, -1)                                       # -inf: no key
+        p = torch.where(vis[:, None, :], torch.exp(sm - lse[..., None]), torch.zeros(()))
+        o = torch.einsum("thl,ld->thd", p, torch.from_numpy(vf[0]))
+        cand = pos[None, :] <= (i - window)[:, None]
+        sc = torch.exp(s - torch.from_numpy(lse_in)[..., None]).sum(1)
+        sc = torch.where(cand, sc, torch.zeros(()))
+        assert np.array_equal(np.isneginf(sl["lse"]), np.isneginf(lse.numpy()))
+        fin = np.isfinite(lse.numpy())
+        assert np.allclose(sl["lse"][fin], lse.numpy()[fin], rtol=1e-13)
+        assert np.allclose(sl["o"], o.numpy(), rtol=1e-11, atol=1e-14)
+        assert np.allclose(sl["score"], sc.numpy(), rtol=1e-11, atol=1e-15)
+
+
 # -------------------------------------------------- block-level selection --
 def check_select_blocks_of_one_are_token_level():
     # blocks of a single position are the token-level selection (pinned above
@@ -355,4 +397,5 @@ ALL_CHECKS = [
     check_all_equal_keys, check_sparse_equals_dense, check_sparse_vs_torch,
     check_golden_worked_example, check_select_blocks_of_one_are_token_level,
     check_select_blocks_bruteforce_rank, check_golden_worked_block_selection,
+    check_slice_of_the_whole_cache_is_full_attention, check_slice_vs_torch,
 ]

@@ -52,6 +52,10 @@ MUTANTS = {
                                    "return a > b;  // equal sums: the lower block first"),
     "boundary_block_overlaps_window": ("for (int64_t j = b * block; j < std::min<int64_t>((b + 1) * block, last + 1); ++j)",
                                        "for (int64_t j = b * block; j < (b + 1) * block; ++j)"),
+    "slice_sees_one_key_too_many": ("const int64_t n = std::max<int64_t>(0, std::min<int64_t>(L_slice, i + 1));",
+                                    "const int64_t n = std::max<int64_t>(0, std::min<int64_t>(L_slice, i + 2));"),
+    "slice_score_ignores_given_lse": ("const double ref = lse_in ? lse_in[(size_t)bt * H + h] : lse_row[h];",
+                                      "const double ref = lse_row[h];"),
 }
 
 
