@@ -144,6 +144,115 @@ HS2_API hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, i
                                 hs2_stream_t stream);
 
 /*
+ * hs2_full_attn_select_blocks -- hs2_full_attn_select with the block-level
+ * selection of the HySparse generation before HySparse2, for comparison with
+ * the token-level selection (dpshk.com explainer, section 03: history chosen
+ * in blocks of 64 tokens, so a block with one useful token takes the budget
+ * of 64; cnyes.com article, section "檢索精確到token": the ablation keeps the
+ * same budget and compares the two granularities).
+ *
+ * O and lse are those of hs2_full_attn_select.  Selection (readings of this
+ * library where the pages are silent): candidates C = {0 .. i-window} as for
+ * tokens; block b = positions b*block .. b*block+block-1, a candidate when it
+ * holds a candidate position; its score is the sum of score_j over its
+ * candidate positions; the topk/block blocks of largest score are kept, ties
+ * to the lower block; S = their candidate positions union the window,
+ * ascending in idx[b][t][0 .. n_sel), then -1.  When no more than topk/block
+ * blocks are candidates, S = {0 .. i}.  |S| <= topk + window.
+ * Arguments, layouts, workspace (hs2_full_attn_select_workspace) and status
+ * codes are those of hs2_full_attn_select, plus: block >= 1 and topk a
+ * multiple of block (else HS2_ERR_INVALID_ARG); at most 49152 candidate blocks
+ * per query, (L - window) / block + 1 <= 49152 (else HS2_ERR_UNSUPPORTED).
+ */
+HS2_API hs2_status hs2_full_attn_select_blocks(const void* Q, const hs2_kv_cache* kv, int B, int T,
+                                               int64_t L, int H, int D, float scale, int topk,
+                                               int window, int block, hs2_kv_dtype dt, float* O,
+                                               float* lse, int32_t* idx, int32_t* n_sel,
+                                               void* workspace, size_t workspace_bytes,
+                                               hs2_stream_t stream);
+
+/*
+ * Context parallelism of the full-attention layer and its selection: G ranks
+ * (one per GPU) each hold a contiguous slice of every sequence's cache, L_r
+ * positions starting at global position a_r, and all T queries (query t at
+ * global position q_pos0 + t; a slice-relative position q_pos0 + t - a_r).  The
+ * pages analyse contexts of a million tokens (dpshk.com explainer, section 05;
+ * cnyes.com article, cost paragraph), where one layer's cache spans devices.
+ * One layer is, on every rank:
+ *   1. hs2_cp_attn_partial   -> O_r (normalised over the slice), lse_r
+ *   2. all-gather of lse_r, hs2_cp_lse_combine -> lse (global normaliser)
+ *   3. hs2_cp_rescale(O_r), sum all-reduce of O_r across ranks -> O
+ *   4. hs2_cp_select_local   -> the slice's top-k candidates and their scores
+ *   5. all-gather of the candidate lists, hs2_cp_merge_select -> idx, n_sel
+ * The results equal hs2_full_attn_select on the whole cache (same readings):
+ * the global top-k lies in the union of the slices' top-k lists, and the
+ * merge keeps ties at the lower position.  The collectives are the caller's
+ * (NCCL through torch.distributed in the Python package).  Supported: D ==
+ * 128, H in {8, 16, 32}, B * L_r < 2^31; T may exceed L_r.
+ *
+ * Workspace bytes of hs2_cp_attn_partial / hs2_cp_select_local on one slice;
+ * 0 for arguments they would reject.
+ */
+HS2_API size_t hs2_cp_workspace(int B, int T, int64_t L_local, int H, int D, int topk, int window,
+                                hs2_kv_dtype dt);
+
+/*
+ * Step 1 on one slice: kv holds the slice, K/V [B][L_local][D]; q_pos_local is
+ * query 0's slice-relative position (global position - a_r; it may be
+ * negative or >= L_local).  Key j of the slice is visible to query t when
+ * j <= q_pos_local + t.  Writes O fp32 [B][T][H][D] (normalised over the
+ * visible keys of the slice; 0 where none is visible) and lse fp32 [B][T][H]
+ * (natural log; -inf where none is visible).
+ */
+HS2_API hs2_status hs2_cp_attn_partial(const void* Q, const hs2_kv_cache* kv, int B, int T,
+                                       int64_t L_local, int64_t q_pos_local, int H, int D,
+                                       float scale, hs2_kv_dtype dt, float* O, float* lse,
+                                       void* workspace, size_t workspace_bytes,
+                                       hs2_stream_t stream);
+
+/*
+ * Step 2: lse[e] = log sum_r exp(lse_parts[r * n + e]) for e < n (lse_parts
+ * fp32 [G][n], -inf entries contribute nothing).
+ */
+HS2_API hs2_status hs2_cp_lse_combine(const float* lse_parts, int G, int64_t n, float* lse,
+                                      hs2_stream_t stream);
+
+/*
+ * Step 3 (before the sum across ranks): O_part[e][d] *= exp(lse_part[e] -
+ * lse[e]) for the n rows of D values (0 where lse_part is -inf).
+ */
+HS2_API hs2_status hs2_cp_rescale(float* O_part, const float* lse_part, const float* lse,
+                                  int64_t n, int D, hs2_stream_t stream);
+
+/*
+ * Step 4 on one slice: with lse the global normaliser (step 2's output,
+ * [B][T][H]), score_j = sum_h exp(s_hj - lse_h) for the slice's candidates
+ * (slice-relative j <= q_pos_local + t - window, j < L_local), and the slice's
+ * top-k of them by (score descending, position ascending): cand_idx int32
+ * [B][T][topk] global positions (slice position + key_pos0, key_pos0 = a_r),
+ * ascending, -1 padded; cand_score fp32 [B][T][topk] their scores (-1 for
+ * padding).  topk >= 1.
+ */
+HS2_API hs2_status hs2_cp_select_local(const void* Q, const hs2_kv_cache* kv, int B, int T,
+                                       int64_t L_local, int64_t q_pos_local, int64_t key_pos0,
+                                       int H, int D, float scale, int topk, int window,
+                                       hs2_kv_dtype dt, const float* lse, float* cand_score,
+                                       int32_t* cand_idx, void* workspace,
+                                       size_t workspace_bytes, hs2_stream_t stream);
+
+/*
+ * Step 5: from the G ranks' candidate lists in rank order (cand_score fp32,
+ * cand_idx int32, both [G][B][T][topk]; the ranks' slices ascend), the global
+ * selection of hs2_full_attn_select: the top-k by (score descending, position
+ * ascending), then the window of query position q_pos0 + t, in idx int32
+ * [B][T][topk + window] ascending (-1 padded) and n_sel int32 [B][T].
+ * G * topk <= 51200.
+ */
+HS2_API hs2_status hs2_cp_merge_select(const float* cand_score, const int32_t* cand_idx, int G,
+                                       int B, int T, int64_t q_pos0, int topk, int window,
+                                       int32_t* idx, int32_t* n_sel, hs2_stream_t stream);
+
+/*
  * hs2_sparse_attn -- a sparse-attention layer with KV Reuse (IT Home
  * announcement, "KV Reuse" paragraph: the sparse layers reuse the full
  * layer's KV cache and selection indices; the SWA branch is folded into the

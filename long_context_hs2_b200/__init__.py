@@ -26,7 +26,9 @@ _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error",
 EXPORTED = ("hs2_bridge_kv", "hs2_full_attn_select_workspace", "hs2_full_attn_select",
             "hs2_full_attn_select_noalloc", "hs2_sparse_attn", "hs2_last_device_status",
             "hs2_status_string", "hs2_version", "hs2_set_stage_events",
-            "hs2_set_fault_injection")
+            "hs2_set_fault_injection", "hs2_full_attn_select_blocks", "hs2_cp_workspace",
+            "hs2_cp_attn_partial", "hs2_cp_lse_combine", "hs2_cp_rescale", "hs2_cp_select_local",
+            "hs2_cp_merge_select")
 
 # Size of the scratch area built into the library for hs2_full_attn_select_noalloc.
 HS2_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -69,6 +71,23 @@ def load_library(path: str = LIB_PATH):
     lib.hs2_full_attn_select.restype = i32
     lib.hs2_full_attn_select.argtypes = [P, KV, i32, i32, i64, i32, i32, ctypes.c_float, i32, i32,
                                          i32, P, P, P, P, P, sz, P]
+    lib.hs2_full_attn_select_blocks.restype = i32
+    lib.hs2_full_attn_select_blocks.argtypes = [P, KV, i32, i32, i64, i32, i32, ctypes.c_float,
+                                                i32, i32, i32, i32, P, P, P, P, P, sz, P]
+    lib.hs2_cp_workspace.restype = sz
+    lib.hs2_cp_workspace.argtypes = [i32, i32, i64, i32, i32, i32, i32, i32]
+    lib.hs2_cp_attn_partial.restype = i32
+    lib.hs2_cp_attn_partial.argtypes = [P, KV, i32, i32, i64, i64, i32, i32, ctypes.c_float, i32,
+                                        P, P, P, sz, P]
+    lib.hs2_cp_lse_combine.restype = i32
+    lib.hs2_cp_lse_combine.argtypes = [P, i32, i64, P, P]
+    lib.hs2_cp_rescale.restype = i32
+    lib.hs2_cp_rescale.argtypes = [P, P, P, i64, i32, P]
+    lib.hs2_cp_select_local.restype = i32
+    lib.hs2_cp_select_local.argtypes = [P, KV, i32, i32, i64, i64, i64, i32, i32, ctypes.c_float,
+                                        i32, i32, i32, P, P, P, P, sz, P]
+    lib.hs2_cp_merge_select.restype = i32
+    lib.hs2_cp_merge_select.argtypes = [P, P, i32, i32, i32, i64, i32, i32, P, P, P]
     lib.hs2_full_attn_select_noalloc.restype = i32
     lib.hs2_full_attn_select_noalloc.argtypes = [P, KV, i32, i32, i64, i32, i32, ctypes.c_float,
                                                  i32, i32, i32, P, P, P, P, P]
@@ -149,6 +168,17 @@ def hs2_full_attn_select(Q, kv: hs2_kv_cache, B, T, L, H, D, scale, topk, window
         int(workspace_bytes), _stream(stream)))
 
 
+def hs2_full_attn_select_blocks(Q, kv: hs2_kv_cache, B, T, L, H, D, scale, topk, window, block,
+                                dt, O, lse, idx, n_sel, workspace, workspace_bytes: int,
+                                stream=None):
+    """hs2_full_attn_select with the block-level selection (blocks of `block`
+    positions, topk/block of them kept) instead of the token-level one."""
+    _check("hs2_full_attn_select_blocks", load_library().hs2_full_attn_select_blocks(
+        _ptr(Q), ctypes.byref(kv), int(B), int(T), int(L), int(H), int(D), float(scale),
+        int(topk), int(window), int(block), int(dt), _ptr(O), _ptr(lse), _ptr(idx), _ptr(n_sel),
+        _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
 def hs2_full_attn_select_noalloc(Q, kv: hs2_kv_cache, B, T, L, H, D, scale, topk, window, dt,
                                  O, lse, idx, n_sel, stream=None):
     """hs2_full_attn_select without a workspace argument, for callers that cannot
@@ -183,3 +213,44 @@ def hs2_set_fault_injection(extra_arrivals: int = 0, wait_limit_ns: int = 0):
     With no arguments, restores the defaults."""
     _check("hs2_set_fault_injection",
            load_library().hs2_set_fault_injection(int(extra_arrivals), int(wait_limit_ns)))
+
+
+# ------------------------------------------------ context parallelism --
+def hs2_cp_workspace(B, T, L_local, H, D, topk, window, dt) -> int:
+    return int(load_library().hs2_cp_workspace(int(B), int(T), int(L_local), int(H), int(D),
+                                                int(topk), int(window), int(dt)))
+
+
+def hs2_cp_attn_partial(Q, kv: hs2_kv_cache, B, T, L_local, q_pos_local, H, D, scale, dt, O, lse,
+                        workspace, workspace_bytes: int, stream=None):
+    _check("hs2_cp_attn_partial", load_library().hs2_cp_attn_partial(
+        _ptr(Q), ctypes.byref(kv), int(B), int(T), int(L_local), int(q_pos_local), int(H), int(D),
+        float(scale), int(dt), _ptr(O), _ptr(lse), _ptr(workspace), int(workspace_bytes),
+        _stream(stream)))
+
+
+def hs2_cp_lse_combine(lse_parts, G, n, lse, stream=None):
+    _check("hs2_cp_lse_combine", load_library().hs2_cp_lse_combine(
+        _ptr(lse_parts), int(G), int(n), _ptr(lse), _stream(stream)))
+
+
+def hs2_cp_rescale(O_part, lse_part, lse, n, D, stream=None):
+    _check("hs2_cp_rescale", load_library().hs2_cp_rescale(
+        _ptr(O_part), _ptr(lse_part), _ptr(lse), int(n), int(D), _stream(stream)))
+
+
+def hs2_cp_select_local(Q, kv: hs2_kv_cache, B, T, L_local, q_pos_local, key_pos0, H, D, scale,
+                        topk, window, dt, lse, cand_score, cand_idx, workspace,
+                        workspace_bytes: int, stream=None):
+    _check("hs2_cp_select_local", load_library().hs2_cp_select_local(
+        _ptr(Q), ctypes.byref(kv), int(B), int(T), int(L_local), int(q_pos_local), int(key_pos0),
+        int(H), int(D), float(scale), int(topk), int(window), int(dt), _ptr(lse),
+        _ptr(cand_score), _ptr(cand_idx), _ptr(workspace), int(workspace_bytes),
+        _stream(stream)))
+
+
+def hs2_cp_merge_select(cand_score, cand_idx, G, B, T, q_pos0, topk, window, idx, n_sel,
+                        stream=None):
+    _check("hs2_cp_merge_select", load_library().hs2_cp_merge_select(
+        _ptr(cand_score), _ptr(cand_idx), int(G), int(B), int(T), int(q_pos0), int(topk),
+        int(window), _ptr(idx), _ptr(n_sel), _stream(stream)))

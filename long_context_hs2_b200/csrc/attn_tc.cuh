@@ -262,6 +262,7 @@ __device__ __forceinline__ void tc_partial_setup(uint8_t* smem) {
 // columns each beside the 32 of O^T: all 512 columns).
 constexpr int kTcRetainTiles = 15;
 
+
 // The partial pass of one (group, split) work item: every role's work, with
 // the barriers of tc_partial_setup initialised and the TMEM columns at `tmem`
 // (4N; 512 when RETAIN).  TMEM layout: S^T double buffer at columns 0 and N,
@@ -303,9 +304,9 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
   const int b = grp / p.groups_per_seq;
   const int t0 = (grp % p.groups_per_seq) * G;
   const int t_last = min(p.T, t0 + G) - 1;
-  const long long i_last = p.L - p.T + t_last;
+  const long long i_last = p.qpos0 + t_last;
   const long long k_lo = (long long)split * p.split_keys;
-  const long long k_hi = min(k_lo + p.split_keys, i_last + 1);
+  const long long k_hi = min(min(k_lo + p.split_keys, i_last + 1), p.L);
   const long long part = (long long)grp * p.n_splits + split;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -458,11 +459,11 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
       failed |= !mbar_wait(&s_full[bb], (n >> 1) & 1);
       tc_fence_after();
       // a tile is "full" when every key is in range and causal for every query
-      const bool full_tile = key0 + kTcKeys <= k_hi && key0 + kTcKeys - 1 <= p.L - p.T + t0;
+      const bool full_tile = key0 + kTcKeys <= k_hi && key0 + kTcKeys - 1 <= p.qpos0 + t0;
       // limit[q]: last key query q of the group may see (in range of this split)
       long long limit[G];
 #pragma unroll
-      for (int q = 0; q < G; ++q) limit[q] = min(k_hi - 1, p.L - p.T + t0 + q);
+      for (int q = 0; q < G; ++q) limit[q] = min(k_hi - 1, p.qpos0 + t0 + q);
       const uint32_t s_addr = tmem + lane_base + s_col(n) + c0;
       // kHold (NC <= 16): this key's logits of the warp's rows are loaded once and
       // kept for both sweeps; wider rows reload 16 columns at a time (registers)
@@ -756,7 +757,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   const int b = grp / p.groups_per_seq;
   const int t0 = (grp % p.groups_per_seq) * G;
   const int t_last = min(p.T, t0 + G) - 1;
-  const long long i_last = p.L - p.T + t_last;
+  const long long i_last = p.qpos0 + t_last;
   const long long k_lo = (long long)split * p.split_keys;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -915,7 +916,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
 #pragma unroll
         for (int q = 0; q < G; ++q) {
           const int t = t0 + q;
-          const bool cand = t < p.T && j <= p.L - p.T + t - p.window;
+          const bool cand = t < p.T && j <= p.qpos0 + t - p.window;
           if (cand) {
             p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
             if (p.fuse_select) seg[q * p.split_keys + (int)(j - k_lo)] = acc[q];
@@ -974,7 +975,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     unsigned* h = reinterpret_cast<unsigned*>(smem + SM::kSelWorkOff);    // 2048 counters
     int* off_s = reinterpret_cast<int*>(smem + SM::kSelWorkOff + 8192);   // [ns + 1] list offsets
     auto row_of = [&](int q) { return (long long)b * p.T + t0 + q; };
-    auto nc_of = [&](int q) { return p.L - p.T + t0 + q - p.window + 1; };
+    auto nc_of = [&](int q) { return p.qpos0 + t0 + q - p.window + 1; };
     auto active = [&](int q) { return t0 + q < p.T && nc_of(q) > p.topk && p.topk > 0; };
     auto nseg_of = [&](int q) {
       return (int)max(0LL, min((long long)p.split_keys, nc_of(q) - k_lo));
@@ -1139,7 +1140,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       }
     if (split == 0)  // window, padding and count; or every position when all are taken
       for (int q = 0; q < G && t0 + q < p.T; ++q) {
-        const long long i = p.L - p.T + t0 + q;
+        const long long i = p.qpos0 + t0 + q;
         int32_t* out = p.idx + row_of(q) * p.slots;
         if (nc_of(q) <= p.topk) {
           for (int j = threadIdx.x; j < p.slots; j += kThreads) out[j] = j <= i ? (int32_t)j : -1;
@@ -1188,10 +1189,10 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
   const int b = grp / p.groups_per_seq;
   const int t0 = (grp % p.groups_per_seq) * G;
   const int t_last = min(p.T, t0 + G) - 1;
-  const long long i_last = p.L - p.T + t_last;
+  const long long i_last = p.qpos0 + t_last;
   const long long k_lo = (long long)split * p.score_keys;
-  const long long k_hi = min(k_lo + p.score_keys, i_last - p.window + 1);
-  const int n_tiles = k_lo < k_hi ? (int)((k_hi - k_lo + kTcKeys - 1) / kTcKeys) : 0;
+  const long long k_hi = min(min(k_lo + p.score_keys, i_last - p.window + 1), p.L);
+  const int n_tiles = (!p.no_score && k_lo < k_hi) ? (int)((k_hi - k_lo + kTcKeys - 1) / kTcKeys) : 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ns = p.n_splits;
 
@@ -1278,7 +1279,7 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
     }
-    {
+    if (!p.lse_in) {
       const float2* ml_g = p.part_ml + (long long)grp * ns * N;
       for (int u = st; u < N * ns; u += 128) {
         const int sp = u / N, r = u % N;
@@ -1288,6 +1289,11 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
     for (int u = st; u < G * kHistBins; u += 128) hist_s[u] = 0u;
     softmax_sync<128>();
     for (int r = st; r < N; r += 128) {
+      if (p.lse_in) {  // the normaliser over the whole context (context-parallel slice)
+        const int t = t0 + r / kH;
+        lse2_s[r] = t < p.T ? p.lse_in[((long long)b * p.T + t) * p.H + r % kH] * kLog2e : 0.f;
+        continue;
+      }
       float M = kNegInf;
       for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, ml_s[r * ns + sp].x);
       float lt = 0.f;
@@ -1335,7 +1341,9 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
 #pragma unroll
       for (int q = 0; q < G; ++q) {
         const int t = t0 + q;
-        const bool cand = t < p.T && j <= p.L - p.T + t - p.window;
+        // a candidate lies inside this split (and the cache: a context-parallel
+        // slice may end before the query's candidates do)
+        const bool cand = t < p.T && j < k_hi && j <= p.qpos0 + t - p.window;
         if (cand) p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
         hist_inc(hist_s + q * kHistBins, __float_as_uint(acc[q]) >> kHistShift, cand);
       }
@@ -1347,8 +1355,9 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
       if (cnt && t < p.T) atomicAdd(&p.hist[((long long)b * p.T + t) * kHistBins + (u % kHistBins)], cnt);
     }
     // ---- O and lse of row r, merged by the CTA whose score-split index is r mod
-    //      score_splits: thread st owns element d = st of the row
-    for (int r = split; r < N; r += p.score_splits) {
+    //      score_splits: thread st owns element d = st of the row (not with a
+    //      given normaliser: O and lse were produced by the slice's first pass)
+    for (int r = split; r < N && !p.lse_in; r += p.score_splits) {
       const int t = t0 + r / kH;
       if (t >= p.T) continue;
       const float l2 = lse2_s[r];

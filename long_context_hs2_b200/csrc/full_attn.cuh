@@ -53,6 +53,14 @@ struct FullAttnParams {
   // group's CTA count (non-zero only under fault injection)
   unsigned long long wait_limit_ns;
   unsigned barrier_extra;
+  // query t sits at local key position qpos0 + t (L - T when the cache holds
+  // the whole context; with a context-parallel slice, the queries' position
+  // relative to the slice's first key, which may exceed L)
+  long long qpos0;
+  // context-parallel score pass: the global natural-log normaliser [B][T][H]
+  // replaces the merge of this slice's partials (O and lse are not written)
+  const float* lse_in;
+  int no_score;   // merge the partials into O and lse only (no score pass)
 };
 
 template <int D, bool FP8>
@@ -134,9 +142,9 @@ __global__ void __launch_bounds__(160) attn_partial_kernel(const __grid_constant
   const int b = grp / p.groups_per_seq;
   const int t0 = (grp % p.groups_per_seq) * p.G;
   const int t_last = min(p.T, t0 + p.G) - 1;
-  const long long i_last = p.L - p.T + t_last;
+  const long long i_last = p.qpos0 + t_last;
   const long long k_lo = (long long)split * p.split_keys;
-  const long long k_hi = min(k_lo + p.split_keys, i_last + 1);
+  const long long k_hi = min(min(k_lo + p.split_keys, i_last + 1), p.L);
   const long long part = (long long)grp * p.n_splits + split;
 
   if (split == 0) {  // clear the group's level-1 selection histograms
@@ -194,7 +202,7 @@ __global__ void __launch_bounds__(160) attn_partial_kernel(const __grid_constant
       const int r = mt * 16 + g + 8 * h;
       const int t = t0 + r / p.H;
       row_ok[mt][h] = t < p.T;
-      i_row[mt][h] = p.L - p.T + t;
+      i_row[mt][h] = p.qpos0 + t;
     }
   const float* ksc = FP8 ? p.k_scale + (long long)b * p.L : nullptr;
   const float* vsc = FP8 ? p.v_scale + (long long)b * p.L : nullptr;
@@ -315,9 +323,9 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
   const int b = grp / p.groups_per_seq;
   const int t0 = (grp % p.groups_per_seq) * G;
   const int t_last = min(p.T, t0 + G) - 1;
-  const long long i_last = p.L - p.T + t_last;
+  const long long i_last = p.qpos0 + t_last;
   const long long k_lo = (long long)split * p.score_keys;
-  const long long k_hi = min(k_lo + p.score_keys, i_last - p.window + 1);
+  const long long k_hi = min(min(k_lo + p.score_keys, i_last - p.window + 1), p.L);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* lse2_s = reinterpret_cast<float*>(smem + SM::kScoreLseOff);
 
@@ -408,7 +416,7 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
       const int tl = r / p.H;
       const int t = t0 + tl;
       qry[mt][h] = tl;
-      i_row[mt][h] = (t < p.T) ? p.L - p.T + t : -1;  // -1: no candidates
+      i_row[mt][h] = (t < p.T) ? p.qpos0 + t : -1;  // -1: no candidates
       lse2[mt][h] = (t < p.T) ? lse2_s[r] : 0.f;
     }
   const float* ksc = FP8 ? p.k_scale + (long long)b * p.L : nullptr;
@@ -489,7 +497,7 @@ __global__ void __launch_bounds__(160) attn_score_kernel(const __grid_constant__
       for (int q = 0; q < G; ++q) {
         const int t = t0 + q;
         if (t >= p.T) break;
-        const long long i_q = p.L - p.T + t;
+        const long long i_q = p.qpos0 + t;
         float* srow = p.score + ((long long)b * p.T + t) * p.L;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)

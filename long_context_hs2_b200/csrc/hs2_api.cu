@@ -10,9 +10,12 @@
 #include <utility>
 
 #include "bridge_gemm.cuh"
+#include "bridge_small.cuh"
+#include "cp.cuh"
 #include "full_attn.cuh"
 #include "attn_tc.cuh"
 #include "select.cuh"
+#include "select_block.cuh"
 #include "sparse_attn.cuh"
 
 using namespace hs2;
@@ -128,10 +131,11 @@ hs2_status check_full_args(const void* Q, const hs2_kv_cache* kv, int B, int T, 
   return HS2_OK;
 }
 
-bool make_full_plan(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt, FullPlan* pl) {
+bool make_full_plan(int B, int T, int64_t L, int H, int D, hs2_kv_dtype dt, FullPlan* pl,
+                    bool allow_fused = true) {
   pl->tc = D == 128;
   pl->rows = pl->tc && H == 32 && T >= 4 ? 128 : 32;
-  pl->fused = pl->tc && pl->rows == 32;
+  pl->fused = allow_fused && pl->tc && pl->rows == 32;
   pl->tile = pl->tc ? kTcKeys : kTile;
   pl->G = pl->rows / H;
   pl->groups_per_seq = (T + pl->G - 1) / pl->G;
@@ -235,7 +239,10 @@ hs2_status run_select(const FullAttnParams& fp, SelectParams sp, cudaStream_t s)
   int cs = 1;
   while (cs < 8 && rows * cs * 2 <= sms) cs *= 2;
   sp.cs = cs;
-  const long long nc_max = std::max<long long>(1, fp.L - fp.window + 1);
+  // the most candidates of any row (a context-parallel slice holds at most L)
+  const long long nc_max =
+      sp.cp ? std::max<long long>(1, std::min<long long>(fp.L, sp.qpos0 + fp.T - fp.window))
+            : std::max<long long>(1, fp.L - fp.window + 1);
   const long long seg = ((nc_max + cs - 1) / cs + 3) / 4 * 4;
   const bool smem = seg <= kSelSmemMax;
   const int bytes = smem ? (int)std::max<long long>(16, seg * 4) : 0;
@@ -246,7 +253,7 @@ hs2_status run_select(const FullAttnParams& fp, SelectParams sp, cudaStream_t s)
 
 template <int D, bool FP8>
 hs2_status run_full(const CUtensorMap& km, const CUtensorMap& vm, const FullAttnParams& fp,
-                    const FullPlan& pl, const SelectParams& sp, cudaStream_t s) {
+                    const FullPlan& pl, cudaStream_t s) {
   using SM = FullAttnSmem<D, FP8>;
   auto kp = attn_partial_kernel<D, FP8>;
   auto ks = fp.G == 1 ? attn_score_kernel<D, FP8, 1>
@@ -257,9 +264,7 @@ hs2_status run_full(const CUtensorMap& km, const CUtensorMap& vm, const FullAttn
                          vm, fp);
   if (st != HS2_OK) return st;
   if (stage_mark(s, false) != cudaSuccess) return HS2_ERR_CUDA;
-  st = launch(ks, dim3(pl.n_groups * pl.score_splits), dim3(160), SM::kScoreBytes, s, 1, km, fp);
-  if (st != HS2_OK) return st;
-  return run_select(fp, sp, s);
+  return launch(ks, dim3(pl.n_groups * pl.score_splits), dim3(160), SM::kScoreBytes, s, 1, km, fp);
 }
 
 template <int N, bool FP8>
@@ -285,18 +290,35 @@ hs2_status run_full_tc(const CUtensorMap& km, const CUtensorMap& vm, const FullA
                 s, 1, km, fp);
 }
 
+// The score kernel alone (a context-parallel slice's second pass: the
+// normaliser comes from fp.lse_in).
+template <int N, bool FP8>
+hs2_status run_score_tc(const CUtensorMap& km, const FullAttnParams& fp, const FullPlan& pl,
+                        cudaStream_t s) {
+  using SM = TcSmem<N, FP8>;
+  auto ks = N == 128 ? attn_tc_score_kernel<N, 4, FP8>
+                     : (fp.G == 1 ? attn_tc_score_kernel<N, 1, FP8>
+                                  : (fp.G == 2 ? attn_tc_score_kernel<N, 2, FP8>
+                                               : attn_tc_score_kernel<N, 4, FP8>));
+  if (!set_smem(ks, SM::kSBytes)) return HS2_ERR_CUDA;
+  return launch(ks, dim3(pl.n_groups * pl.score_splits), dim3(tc_score_threads(FP8)), SM::kSBytes,
+                s, 1, km, fp);
+}
+
 // The fused tcgen05 pass (N = 32): arrival counters cleared, then one
 // cooperative launch (the CTAs of a group wait for one another); the
 // selection runs inside it when a row's candidates fit its shared memory,
 // else as the selection kernel after it.
 template <bool FP8>
 hs2_status run_fused_tc(const CUtensorMap& km, const CUtensorMap& vm, FullAttnParams fp,
-                        const FullPlan& pl, const SelectParams& sp, cudaStream_t s) {
+                        const FullPlan& pl, const SelectParams& sp, bool token_select,
+                        cudaStream_t s) {
   using SM = TcSmem<32, FP8>;
   static_assert(SM::kBytes <= 232448, "shared memory per CTA");
   // the selection is fused when a split's candidate scores of the group's
-  // rows fit the P^T buffers (shared memory free after the partial pass)
-  fp.fuse_select = (long long)fp.G * fp.split_keys * 4 <= SM::kNP * SM::kPBytes &&
+  // rows fit the P^T buffers (shared memory free after the partial pass);
+  // without token_select the caller runs another selection on the scores
+  fp.fuse_select = token_select && (long long)fp.G * fp.split_keys * 4 <= SM::kNP * SM::kPBytes &&
                    pl.n_splits <= 256;
   // the logits of every tile stay in TMEM for the score pass when a split has
   // at most kTcRetainTiles tiles
@@ -317,7 +339,29 @@ hs2_status run_fused_tc(const CUtensorMap& km, const CUtensorMap& vm, FullAttnPa
                                   SM::kBytes, s, 1, pl.n_splits > 1, false, km, vm, fp);
   if (st != HS2_OK) return st;
   if (stage_mark(s, false) != cudaSuccess) return HS2_ERR_CUDA;
-  return fp.fuse_select ? HS2_OK : run_select(fp, sp, s);
+  return (fp.fuse_select || !token_select) ? HS2_OK : run_select(fp, sp, s);
+}
+
+// Block-level selection from the score rows the attention pass wrote.
+hs2_status run_select_blocks(const FullAttnParams& fp, int topk, int window, int block,
+                             int32_t* idx, int32_t* n_sel, cudaStream_t s) {
+  BlockSelectParams bp;
+  bp.score = fp.score;
+  bp.idx = idx;
+  bp.n_sel = n_sel;
+  bp.T = fp.T;
+  bp.L = fp.L;
+  bp.topk = topk;
+  bp.window = window;
+  bp.slots = topk + window;
+  bp.block = block;
+  bp.block_shift = (block & (block - 1)) == 0 ? __builtin_ctz((unsigned)block) : -1;
+  bp.qpos0 = fp.qpos0;
+  const long long nblk_max = std::max<long long>(1, (fp.L - window) / block + 1);
+  const size_t bytes = (size_t)(nblk_max + topk / block) * 4;
+  if (!set_smem(select_blocks_kernel, (int)bytes)) return HS2_ERR_CUDA;
+  return launch(select_blocks_kernel, dim3((unsigned)((long long)fp.B * fp.T)), dim3(kBlkThreads),
+                bytes, s, 1, bp);
 }
 
 template <int MT, int D, bool FP8>
@@ -383,28 +427,28 @@ size_t hs2_full_attn_select_workspace(int B, int T, int64_t L, int H, int D, int
   return pl.total;
 }
 
-hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, int T, int64_t L,
-                                int H, int D, float scale, int topk, int window,
-                                hs2_kv_dtype dt, float* O, float* lse, int32_t* idx,
-                                int32_t* n_sel, void* workspace, size_t workspace_bytes,
-                                hs2_stream_t stream) {
-  const hs2_status chk = check_full_args(Q, kv, B, T, L, H, D, scale, topk, window, dt, O, lse,
-                                         idx, n_sel);
-  if (chk != HS2_OK) return chk;
-  FullPlan pl;
-  make_full_plan(B, T, L, H, D, dt, &pl);
+}  // extern "C"
+
+namespace {
+
+// Plan, tensor maps and kernel parameters of a full-attention call over a
+// cache of L positions (allow_fused: the fused decode kernel may be planned).
+hs2_status setup_full(const void* Q, const hs2_kv_cache* kv, int B, int T, int64_t L, int H, int D,
+                      float scale, int topk, int window, hs2_kv_dtype dt, float* O, float* lse,
+                      int32_t* idx, int32_t* n_sel, void* workspace, size_t workspace_bytes,
+                      bool allow_fused, FullPlan& pl, CUtensorMap& km, CUtensorMap& vm,
+                      FullAttnParams& fp, SelectParams& sp) {
+  make_full_plan(B, T, L, H, D, dt, &pl, allow_fused);
   if (!workspace || workspace_bytes < pl.total || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
 
   const bool fp8 = dt == HS2_KV_FP8_E4M3;
   const int elem = fp8 ? 1 : 2;
-  CUtensorMap km, vm;
   const uint32_t box_cols = fp8 ? 128u : 64u;
   if (!make_map_2d(&km, kv->k, (uint64_t)B * L, D, elem, box_cols, pl.tile) ||
       !make_map_2d(&vm, kv->v, (uint64_t)B * L, D, elem, box_cols, pl.tile))
     return HS2_ERR_CUDA;
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  FullAttnParams fp;
   fp.q = static_cast<const __nv_bfloat16*>(Q);
   fp.k_scale = fp8 ? kv->k_scale : nullptr;
   fp.v_scale = fp8 ? kv->v_scale : nullptr;
@@ -429,7 +473,6 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
   fp.window = window;
   fp.scale_log2 = scale * kLog2e;
 
-  SelectParams sp;
   sp.score = fp.score;
   sp.hist = fp.hist;
   sp.idx = idx;
@@ -451,21 +494,214 @@ hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, in
   fp.fuse_select = 0;
   fp.wait_limit_ns = t_wait_limit_ns;
   fp.barrier_extra = t_barrier_extra;
+  fp.qpos0 = L - T;
+  fp.lse_in = nullptr;
+  fp.no_score = 0;
+  sp.qpos0 = L - T;
+  sp.cp = 0;
+  sp.key_off = 0;
+  sp.cand_score = nullptr;
+  return HS2_OK;
+}
+
+// The full-attention pass, then the token-level selection (sel_block == 0) or
+// the block-level selection with blocks of sel_block positions.
+hs2_status full_attn_select_impl(const void* Q, const hs2_kv_cache* kv, int B, int T, int64_t L,
+                                 int H, int D, float scale, int topk, int window, int sel_block,
+                                 hs2_kv_dtype dt, float* O, float* lse, int32_t* idx,
+                                 int32_t* n_sel, void* workspace, size_t workspace_bytes,
+                                 hs2_stream_t stream) {
+  const hs2_status chk = check_full_args(Q, kv, B, T, L, H, D, scale, topk, window, dt, O, lse,
+                                         idx, n_sel);
+  if (chk != HS2_OK) return chk;
+  FullPlan pl;
+  CUtensorMap km, vm;
+  FullAttnParams fp;
+  SelectParams sp;
+  const hs2_status su = setup_full(Q, kv, B, T, L, H, D, scale, topk, window, dt, O, lse, idx,
+                                   n_sel, workspace, workspace_bytes, true, pl, km, vm, fp, sp);
+  if (su != HS2_OK) return su;
+  const bool fp8 = dt == HS2_KV_FP8_E4M3;
 
   cudaStream_t s = (cudaStream_t)stream;
-  if (pl.fused)
-    return fp8 ? run_fused_tc<true>(km, vm, fp, pl, sp, s) : run_fused_tc<false>(km, vm, fp, pl, sp, s);
-  if (pl.tc) {
-    const hs2_status st =
-        fp8 ? (pl.rows == 128 ? run_full_tc<128, true>(km, vm, fp, pl, s)
-                              : run_full_tc<32, true>(km, vm, fp, pl, s))
-            : (pl.rows == 128 ? run_full_tc<128, false>(km, vm, fp, pl, s)
-                              : run_full_tc<32, false>(km, vm, fp, pl, s));
+  const bool token = sel_block == 0;
+  hs2_status st;
+  if (pl.fused) {
+    st = fp8 ? run_fused_tc<true>(km, vm, fp, pl, sp, token, s)
+             : run_fused_tc<false>(km, vm, fp, pl, sp, token, s);
+    if (st != HS2_OK || token) return st;
+  } else {
+    if (pl.tc)
+      st = fp8 ? (pl.rows == 128 ? run_full_tc<128, true>(km, vm, fp, pl, s)
+                                 : run_full_tc<32, true>(km, vm, fp, pl, s))
+               : (pl.rows == 128 ? run_full_tc<128, false>(km, vm, fp, pl, s)
+                                 : run_full_tc<32, false>(km, vm, fp, pl, s));
+    else  // head_dim 64 (bf16 only): the mma.sync kernels
+      st = run_full<64, false>(km, vm, fp, pl, s);
     if (st != HS2_OK) return st;
-    return run_select(fp, sp, s);
+    if (token) return run_select(fp, sp, s);
   }
-  // head_dim 64 (bf16 only): the mma.sync kernels
-  return run_full<64, false>(km, vm, fp, pl, sp, s);
+  return run_select_blocks(fp, topk, window, sel_block, idx, n_sel, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+hs2_status hs2_full_attn_select(const void* Q, const hs2_kv_cache* kv, int B, int T, int64_t L,
+                                int H, int D, float scale, int topk, int window,
+                                hs2_kv_dtype dt, float* O, float* lse, int32_t* idx,
+                                int32_t* n_sel, void* workspace, size_t workspace_bytes,
+                                hs2_stream_t stream) {
+  return full_attn_select_impl(Q, kv, B, T, L, H, D, scale, topk, window, 0, dt, O, lse, idx,
+                               n_sel, workspace, workspace_bytes, stream);
+}
+
+hs2_status hs2_full_attn_select_blocks(const void* Q, const hs2_kv_cache* kv, int B, int T,
+                                       int64_t L, int H, int D, float scale, int topk,
+                                       int window, int block, hs2_kv_dtype dt, float* O,
+                                       float* lse, int32_t* idx, int32_t* n_sel,
+                                       void* workspace, size_t workspace_bytes,
+                                       hs2_stream_t stream) {
+  if (block < 1 || topk < 0 || topk % block != 0) return HS2_ERR_INVALID_ARG;
+  const hs2_status chk = check_full_args(Q, kv, B, T, L, H, D, scale, topk, window, dt, O, lse,
+                                         idx, n_sel);
+  if (chk != HS2_OK) return chk;
+  if ((L - window) / block + 1 > kBlkMaxBlocks) return HS2_ERR_UNSUPPORTED;
+  return full_attn_select_impl(Q, kv, B, T, L, H, D, scale, topk, window, block, dt, O, lse, idx,
+                               n_sel, workspace, workspace_bytes, stream);
+}
+
+// ------------------------------------------------ context parallelism --
+size_t hs2_cp_workspace(int B, int T, int64_t L_local, int H, int D, int topk, int window,
+                        hs2_kv_dtype dt) {
+  if (!check_attn_shape(B, 1, L_local, H, D, dt) || T < 1 || D != 128 || topk < 0 ||
+      window < 1 || topk + window > 4096)
+    return 0;
+  FullPlan pl;
+  make_full_plan(B, T, L_local, H, D, dt, &pl, false);
+  return pl.total;
+}
+
+// Shared checks of the two per-slice calls; T may exceed L_local (a slice can
+// be shorter than the chunk of queries).
+static hs2_status check_cp_slice(const void* Q, const hs2_kv_cache* kv, int B, int T,
+                                 int64_t L_local, int64_t q_pos_local, int H, int D, float scale,
+                                 hs2_kv_dtype dt) {
+  if (!Q || !kv || !kv->k || !kv->v || !aligned16(Q) || !aligned16(kv->k) || !aligned16(kv->v))
+    return HS2_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || L_local < 1 || !std::isfinite(scale)) return HS2_ERR_INVALID_ARG;
+  if (q_pos_local < -(int64_t)T || q_pos_local > ((int64_t)1 << 40)) return HS2_ERR_INVALID_ARG;
+  if (dt == HS2_KV_FP8_E4M3 && (!kv->k_scale || !kv->v_scale || !aligned4(kv->k_scale) ||
+                                !aligned4(kv->v_scale)))
+    return HS2_ERR_INVALID_ARG;
+  if (!check_attn_shape(B, 1, L_local, H, D, dt) || D != 128) return HS2_ERR_UNSUPPORTED;
+  return HS2_OK;
+}
+
+hs2_status hs2_cp_attn_partial(const void* Q, const hs2_kv_cache* kv, int B, int T,
+                               int64_t L_local, int64_t q_pos_local, int H, int D, float scale,
+                               hs2_kv_dtype dt, float* O, float* lse, void* workspace,
+                               size_t workspace_bytes, hs2_stream_t stream) {
+  hs2_status st = check_cp_slice(Q, kv, B, T, L_local, q_pos_local, H, D, scale, dt);
+  if (st != HS2_OK) return st;
+  if (!O || !lse || !aligned16(O) || !aligned4(lse)) return HS2_ERR_INVALID_ARG;
+  FullPlan pl;
+  CUtensorMap km, vm;
+  FullAttnParams fp;
+  SelectParams sp;
+  st = setup_full(Q, kv, B, T, L_local, H, D, scale, 0, 1, dt, O, lse, nullptr, nullptr,
+                  workspace, workspace_bytes, false, pl, km, vm, fp, sp);
+  if (st != HS2_OK) return st;
+  fp.qpos0 = q_pos_local;
+  fp.no_score = 1;
+  const bool fp8 = dt == HS2_KV_FP8_E4M3;
+  cudaStream_t s = (cudaStream_t)stream;
+  return fp8 ? (pl.rows == 128 ? run_full_tc<128, true>(km, vm, fp, pl, s)
+                               : run_full_tc<32, true>(km, vm, fp, pl, s))
+             : (pl.rows == 128 ? run_full_tc<128, false>(km, vm, fp, pl, s)
+                               : run_full_tc<32, false>(km, vm, fp, pl, s));
+}
+
+hs2_status hs2_cp_select_local(const void* Q, const hs2_kv_cache* kv, int B, int T,
+                               int64_t L_local, int64_t q_pos_local, int64_t key_pos0, int H,
+                               int D, float scale, int topk, int window, hs2_kv_dtype dt,
+                               const float* lse, float* cand_score, int32_t* cand_idx,
+                               void* workspace, size_t workspace_bytes, hs2_stream_t stream) {
+  hs2_status st = check_cp_slice(Q, kv, B, T, L_local, q_pos_local, H, D, scale, dt);
+  if (st != HS2_OK) return st;
+  if (!lse || !cand_score || !cand_idx || !aligned4(lse) || !aligned4(cand_score) ||
+      !aligned4(cand_idx) || topk < 1 || window < 1 || topk + window > 4096 || key_pos0 < 0 ||
+      key_pos0 + L_local > INT32_MAX)
+    return HS2_ERR_INVALID_ARG;
+  FullPlan pl;
+  CUtensorMap km, vm;
+  FullAttnParams fp;
+  SelectParams sp;
+  st = setup_full(Q, kv, B, T, L_local, H, D, scale, topk, window, dt, nullptr, nullptr, cand_idx,
+                  nullptr, workspace, workspace_bytes, false, pl, km, vm, fp, sp);
+  if (st != HS2_OK) return st;
+  fp.qpos0 = q_pos_local;
+  fp.lse_in = lse;
+  sp.qpos0 = q_pos_local;
+  sp.cp = 1;
+  sp.key_off = key_pos0;
+  sp.cand_score = cand_score;
+  sp.slots = topk;
+  const bool fp8 = dt == HS2_KV_FP8_E4M3;
+  cudaStream_t s = (cudaStream_t)stream;
+  // the level-1 selection histograms are cleared by the partial pass, which
+  // this call does not run
+  if (cudaMemsetAsync(fp.hist, 0, (size_t)B * T * kHistBins * 4, s) != cudaSuccess) {
+    cudaGetLastError();
+    return HS2_ERR_CUDA;
+  }
+  st = fp8 ? (pl.rows == 128 ? run_score_tc<128, true>(km, fp, pl, s)
+                             : run_score_tc<32, true>(km, fp, pl, s))
+           : (pl.rows == 128 ? run_score_tc<128, false>(km, fp, pl, s)
+                             : run_score_tc<32, false>(km, fp, pl, s));
+  if (st != HS2_OK) return st;
+  return run_select(fp, sp, s);
+}
+
+hs2_status hs2_cp_lse_combine(const float* lse_parts, int G, int64_t n, float* lse,
+                              hs2_stream_t stream) {
+  if (!lse_parts || !lse || G < 1 || n < 1) return HS2_ERR_INVALID_ARG;
+  const int grid = (int)std::min<int64_t>((n + 255) / 256, 4 * sm_count());
+  return launch(cp_lse_combine_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, 1,
+                lse_parts, G, (long long)n, lse);
+}
+
+hs2_status hs2_cp_rescale(float* O_part, const float* lse_part, const float* lse, int64_t n,
+                          int D, hs2_stream_t stream) {
+  if (!O_part || !lse_part || !lse || n < 1 || D < 1) return HS2_ERR_INVALID_ARG;
+  const int grid = (int)std::min<int64_t>((n * D + 255) / 256, 8 * sm_count());
+  return launch(cp_rescale_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, 1, O_part,
+                lse_part, lse, (long long)n, D);
+}
+
+hs2_status hs2_cp_merge_select(const float* cand_score, const int32_t* cand_idx, int G, int B,
+                               int T, int64_t q_pos0, int topk, int window, int32_t* idx,
+                               int32_t* n_sel, hs2_stream_t stream) {
+  if (!cand_score || !cand_idx || !idx || !n_sel || G < 1 || B < 1 || T < 1 || topk < 1 ||
+      window < 1 || topk + window > 4096 || q_pos0 < 0 || q_pos0 + T > INT32_MAX)
+    return HS2_ERR_INVALID_ARG;
+  if ((int64_t)G * topk * 4 > 200 * 1024) return HS2_ERR_UNSUPPORTED;
+  CpMergeParams p;
+  p.cand_score = cand_score;
+  p.cand_idx = cand_idx;
+  p.idx = idx;
+  p.n_sel = n_sel;
+  p.rows = (long long)B * T;
+  p.G = G;
+  p.T = T;
+  p.topk = topk;
+  p.window = window;
+  p.qpos0 = q_pos0;
+  const int bytes = G * topk * 4;
+  if (!set_smem(cp_merge_select_kernel, bytes)) return HS2_ERR_CUDA;
+  return launch(cp_merge_select_kernel, dim3((unsigned)p.rows), dim3(kCpThreads), (size_t)bytes,
+                (cudaStream_t)stream, 1, p);
 }
 
 hs2_status hs2_sparse_attn(const void* Q, const hs2_kv_cache* kv, int B, int T, int64_t L, int H,
@@ -530,6 +766,30 @@ void fill_bridge_params(BridgeParams* p, const hs2_kv_cache* caches, int n_layer
   p->fp8 = fp8 ? 1 : 0;
 }
 
+// The few-token path of hs2_bridge_kv (T <= kBsMaxT): one cluster of
+// kBsCluster CTAs per 128-column segment, the hidden dimension split over the
+// cluster (bridge_small.cuh).
+hs2_status bridge_small(const void* X, int64_t T, int hidden, const void* Wt, int n_layers,
+                        bool fp8, const hs2_kv_cache* caches, int64_t row_offset,
+                        cudaStream_t s) {
+  const int np = (int)((T + 15) / 16 * 16);
+  CUtensorMap xm, wm;
+  if (!make_map_2d(&xm, X, (uint64_t)T, (uint64_t)hidden, 2, kBrBK, (uint32_t)np) ||
+      !make_map_2d(&wm, Wt, (uint64_t)n_layers * kBrBN, (uint64_t)hidden, 2, kBrBK, 128))
+    return HS2_ERR_CUDA;
+  BridgeParams p;
+  fill_bridge_params(&p, caches, n_layers, fp8, T, row_offset, hidden);
+  auto k = np == 16 ? bridge_small_kernel<16>
+                    : np == 32 ? bridge_small_kernel<32>
+                               : np == 48 ? bridge_small_kernel<48> : bridge_small_kernel<64>;
+  const int bytes = np == 16 ? BsSmem<16>::kBytes
+                             : np == 32 ? BsSmem<32>::kBytes
+                                        : np == 48 ? BsSmem<48>::kBytes : BsSmem<64>::kBytes;
+  if (!set_smem(k, bytes)) return HS2_ERR_CUDA;
+  return launch(k, dim3((unsigned)(n_layers * 2 * kBsCluster)), dim3(kBsThreads), (size_t)bytes, s,
+                kBsCluster, xm, wm, p);
+}
+
 }  // namespace
 
 extern "C" hs2_status hs2_bridge_kv(const void* X, int64_t T, int hidden, const void* Wt,
@@ -549,6 +809,8 @@ extern "C" hs2_status hs2_bridge_kv(const void* X, int64_t T, int hidden, const 
   }
   if (D != 128 || hidden % kBrBK != 0 || n_layers > kBrMaxLayers || T > INT32_MAX - kBrBM)
     return HS2_ERR_UNSUPPORTED;
+  if (T <= kBsMaxT) return bridge_small(X, T, hidden, Wt, n_layers, fp8, caches, cache_row_offset,
+                                        (cudaStream_t)stream);
   CUtensorMap xm, wm;
   if (!make_map_2d(&xm, X, (uint64_t)T, (uint64_t)hidden, 2, kBrBK, kBrBM) ||
       !make_map_2d(&wm, Wt, (uint64_t)n_layers * kBrBN, (uint64_t)hidden, 2, kBrBK, kBrBN))

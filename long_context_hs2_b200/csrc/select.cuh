@@ -32,6 +32,12 @@ struct SelectParams {
   int T;
   long long L;
   int topk, window, slots, cs;
+  long long qpos0;       // query t sits at position qpos0 + t (L - T for a whole cache)
+  // context-parallel slice: only the slice's candidates are selected (no
+  // window), written as global positions (+ key_off) with their scores
+  int cp;
+  long long key_off;
+  float* cand_score;     // [B*T][topk] when cp
 };
 
 __device__ __forceinline__ uint32_t sel_cluster_rank() {
@@ -177,15 +183,24 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
   const uint32_t rank = cs > 1 ? sel_cluster_rank() : 0u;
   const long long row = blockIdx.x / cs;
   const int t = (int)(row % p.T);
-  const long long i = p.L - p.T + t;
-  const long long nc = i - p.window + 1;  // candidates 0 .. nc-1
+  const long long i = p.qpos0 + t;
+  // candidates 0 .. nc-1 (a context-parallel slice holds positions 0 .. L-1 of them)
+  const long long nc = p.cp ? max(0LL, min(i - p.window + 1, p.L)) : i - p.window + 1;
   int32_t* out = p.idx + row * p.slots;
 
-  if (nc <= p.topk) {  // every candidate is taken: S = {0 .. i}
+  if (nc <= p.topk) {  // every candidate is taken: S = {0 .. i}, or the slice's candidates
     if (rank == 0) {
-      const long long n = i + 1;
-      for (long long j = threadIdx.x; j < p.slots; j += kSelThreads) out[j] = j < n ? (int32_t)j : -1;
-      if (threadIdx.x == 0) p.n_sel[row] = (int32_t)n;
+      if (p.cp) {
+        const float* srow = p.score + row * p.L;
+        for (long long j = threadIdx.x; j < p.slots; j += kSelThreads) {
+          out[j] = j < nc ? (int32_t)(j + p.key_off) : -1;
+          p.cand_score[row * p.slots + j] = j < nc ? srow[j] : -1.f;
+        }
+      } else {
+        const long long n = i + 1;
+        for (long long j = threadIdx.x; j < p.slots; j += kSelThreads) out[j] = j < n ? (int32_t)j : -1;
+        if (threadIdx.x == 0) p.n_sel[row] = (int32_t)n;
+      }
     }
     return;  // the same branch for every CTA of the cluster: no cluster barrier follows
   }
@@ -326,7 +341,10 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
       const unsigned selm = __ballot_sync(0xffffffffu, sel);
       if (sel) {
         const int o = pos + __popc(selm & ((1u << lane) - 1u));
-        if (o < p.topk) out[o] = (int32_t)(s0 + j);
+        if (o < p.topk) {
+          out[o] = (int32_t)(s0 + j + p.key_off);
+          if (p.cp) p.cand_score[row * p.slots + o] = __uint_as_float(v);
+        }
       }
       pos += __popc(selm);
       eq_rank += __popc(eqm);
@@ -334,7 +352,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
     if (rank == (uint32_t)(cs - 1) && warp == kSelThreads / 32 - 1 && lane == 0 && pos != p.topk)
       raise_status(kStatusBadIndex);
   }
-  if (rank == 0) {
+  if (rank == 0 && !p.cp) {
     const long long wstart = i - p.window + 1;
     for (int w = threadIdx.x; w < p.window; w += kSelThreads) out[p.topk + w] = (int32_t)(wstart + w);
     for (int s = p.topk + p.window + threadIdx.x; s < p.slots; s += kSelThreads) out[s] = -1;

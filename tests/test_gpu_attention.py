@@ -207,3 +207,30 @@ def test_decode_bf16_unaligned_slot_shares():
     # starts inside a 16-key group and ends on a partly valid one
     _check_block(WORKLOADS["decode_bf16_32k"].resized(L=8192, topk=1000, window=100,
                                                       n_needles=16))
+
+
+@pytest.mark.parametrize("H", [8, 16, 32])
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_sparse_random_index_lists(H, kv):
+    # each query gets its own random set of positions (unsorted, any size from
+    # 0 to the full budget): tiles end anywhere, clusters split them anywhere,
+    # and some queries have no position at all (O = 0)
+    name = "decode_bf16_32k" if kv == "bf16" else "decode_fp8_256k"
+    wl = WORKLOADS[name].resized(B=3, T=4, L=6000, H=H, n_needles=0, n_sparse=1,
+                                 **({"fp8_scale": "mantissa"} if kv == "fp8" else {}))
+    inp = make_attention_inputs(wl, needles=False)
+    di = tl.DeviceInputs(inp)
+    slots = wl.topk + wl.window
+    rng = np.random.default_rng(7 + H)
+    idx = -np.ones((wl.B * wl.T, slots), dtype=np.int32)
+    nsel = np.zeros(wl.B * wl.T, dtype=np.int32)
+    sizes = [0, 1, 127, 128, 129, 700, slots, slots - 1, 300, 16, 1000, 5]
+    for r in range(wl.B * wl.T):
+        n = sizes[r % len(sizes)]
+        idx[r, :n] = rng.choice(wl.L, n, replace=False)
+        nsel[r] = n
+    o_gpu = tl.run_sparse(di, 0, idx, nsel, slots)
+    o_orc = tl.oracle_sparse(inp, 0, idx, nsel)
+    tol = tl.TOL_FP8 if kv == "fp8" else tl.TOL_BF16
+    assert tl.max_abs(o_gpu, o_orc) <= tol
+    assert np.all(o_gpu[nsel == 0] == 0)

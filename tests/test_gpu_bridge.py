@@ -91,7 +91,9 @@ def _check_fp8(gpu, orc, rows_gpu, l, eps):
         g = vals[codes]
         ok = (g >= np.minimum(lo, hi)) & (g <= np.maximum(lo, hi))
         assert ok.all(), (np.argwhere(~ok)[:5], g[~ok][:5], (y / osc[:, None])[~ok][:5])
-        assert (codes != oc).mean() <= 1e-3
+        # every code is valid (above); codes off the oracle's own are the rare
+        # rounding decisions within eps of a midpoint
+        assert (codes != oc).sum() <= max(1, 1e-3 * codes.size)
         deq = P.dec_e4m3(codes, scale)
         assert np.abs(deq - y).max() <= 3e-2
 
@@ -144,3 +146,45 @@ def test_bridge_full_size_sampled_rows(fp8):
             _check_fp8(gpu, orc, rows, l, eps)
         else:
             _check_bf16(gpu, orc, rows, l)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+@pytest.mark.parametrize("T", [1, 7, 33, 64])
+def test_bridge_decode_append_few_tokens(T, fp8):
+    # the decode-time append: T new tokens bridged into all six target layers at
+    # the full hidden size, written at a row offset of an existing cache (the
+    # few-token path: clusters over the hidden dimension); rows outside the
+    # append must be left as they were
+    wl = WORKLOADS["bridge_131k"].resized(T=T, seed=WORKLOADS["bridge_131k"].seed + T)
+    bi = make_bridge_inputs(wl)
+    off, total = 4093, 4093 + T + 5
+    gpu = _run(bi, fp8, row_offset=off, total_rows=total)
+    orc = oracle.bridge(bi.x, bi.wt, wl.n_layers, wl.D)
+    eps = _eps(bi, np.arange(wl.T)) if fp8 else None
+    untouched = np.r_[0:off, off + T:total]
+    for l in range(wl.n_layers):
+        if fp8:
+            _check_fp8(gpu, orc, np.arange(T) + off, l, eps)
+            for kv in (0, 1):
+                assert (gpu[l][kv][untouched] == 0x55).all()
+                assert (gpu[l][2 + kv][untouched] == -1.0).all()
+        else:
+            _check_bf16(gpu, orc, np.arange(T) + off, l)
+            for kv in (0, 1):
+                assert (gpu[l][kv][untouched] == 0x40E0).all()
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_bridge_few_tokens_small_hidden(fp8):
+    # hidden 256 is 4 slices of 64: half of each segment's cluster has no slice
+    # of the hidden dimension and contributes zeros to the reduction
+    wl = WORKLOADS["bridge_131k"].resized(T=5, hidden=256, n_layers=2)
+    bi = make_bridge_inputs(wl)
+    gpu = _run(bi, fp8, row_offset=3, total_rows=11)
+    orc = oracle.bridge(bi.x, bi.wt, wl.n_layers, wl.D)
+    eps = _eps(bi, np.arange(wl.T)) if fp8 else None
+    for l in range(wl.n_layers):
+        if fp8:
+            _check_fp8(gpu, orc, np.arange(wl.T) + 3, l, eps)
+        else:
+            _check_bf16(gpu, orc, np.arange(wl.T) + 3, l)
