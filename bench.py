@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bridge", action="store_true")
     ap.add_argument("--no-configs", action="store_true")
+    ap.add_argument("--only", choices=["append", "blocks", "configs", "decode_fp8_256k",
+                                       "chunk_fp8_1m"], default=None,
+                    help="run one section alone on one GPU and print its JSON (for profiling)")
     return ap.parse_args()
 
 
@@ -265,8 +268,111 @@ def bench_bridge(torch, hs2, args, stream):
     return out
 
 
+def bench_bridge_append(torch, hs2, stream, flush_fn, peak_gbs):
+    """Times the decode-time append of hs2_bridge_kv: T in {1, 64} new tokens
+    bridged into the six target layers (hidden 4096, D = 128) at a row offset of
+    existing caches, L2 flushed before every call.  The call reads the weights
+    once (HBM-bound): algorithmic bytes = Wt + X + the written rows."""
+    from hs2_synth import WORKLOADS as W
+    wl = W["bridge_131k"]
+    hidden, nl, D = wl.hidden, wl.n_layers, wl.D
+    g = torch.Generator(device="cuda").manual_seed(wl.seed)
+    wt = (torch.randn(nl * 2 * D, hidden, device="cuda", generator=g) / 64).to(torch.bfloat16)
+    rows = 4096
+    out = {}
+    for T in (1, 64):
+        x = (torch.randn(T, hidden, device="cuda", generator=g) / 64).to(torch.bfloat16)
+        for name, dt in (("bf16", hs2.HS2_KV_BF16), ("fp8", hs2.HS2_KV_FP8_E4M3)):
+            if dt == hs2.HS2_KV_BF16:
+                bufs = [(torch.empty(rows, D, dtype=torch.bfloat16, device="cuda"),
+                         torch.empty(rows, D, dtype=torch.bfloat16, device="cuda"), None, None)
+                        for _ in range(nl)]
+                row_bytes = 2 * D * 2
+            else:
+                bufs = [(torch.empty(rows, D, dtype=torch.uint8, device="cuda"),
+                         torch.empty(rows, D, dtype=torch.uint8, device="cuda"),
+                         torch.empty(rows, device="cuda"), torch.empty(rows, device="cuda"))
+                        for _ in range(nl)]
+                row_bytes = 2 * (D + 4)
+            caches = [hs2.kv_cache(*b) for b in bufs]
+            for _ in range(3):
+                hs2.hs2_bridge_kv(x, T, hidden, wt, nl, D, dt, caches, 1000, stream)
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(20):
+                flush_fn()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                hs2.hs2_bridge_kv(x, T, hidden, wt, nl, D, dt, caches, 1000, stream)
+                b.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            st = hs2.hs2_last_device_status()
+            if st != 0:
+                raise RuntimeError("bridge append device status: " + hs2.hs2_status_string(st))
+            ms = float(np.median(ts))
+            nbytes = wt.numel() * 2 + x.numel() * 2 + T * nl * row_bytes
+            out["T%d_%s" % (T, name)] = {"us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                                         "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / peak_gbs,
+                                         "algorithmic_bytes": nbytes}
+            del bufs, caches
+    out["workload"] = "T new tokens x hidden 4096 -> 6 layers of K|V (D=128) at a row offset"
+    out["bound"] = "hbm"
+    return out
+
+
+def bench_block_selection(torch, hs2, inp, kv, q, stream, flush_fn):
+    """A/B of the selection granularity on the decode workload's own inputs (the
+    full-attention call alone, L2 flushed before each): token-level selection
+    against the 64-token block-level selection of the earlier HySparse, with the
+    same 1024-position budget; needle recall = share of the planted needles
+    whose position is selected for the query they were planted for."""
+    wl = inp.wl
+    B, T, L, H, D = wl.B, wl.T, wl.L, wl.H, wl.D
+    slots = wl.topk + wl.window
+    dt = hs2.HS2_KV_BF16
+    nb = hs2.hs2_full_attn_select_workspace(B, T, L, H, D, wl.topk, wl.window, dt)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    O = torch.empty(B, T, H, D, device="cuda")
+    idx = torch.empty(B, T, slots, dtype=torch.int32, device="cuda")
+    ns = torch.empty(B, T, dtype=torch.int32, device="cuda")
+    out = {}
+    for label, block in (("token", 0), ("block64", 64)):
+        def call():
+            if block:
+                hs2.hs2_full_attn_select_blocks(q, kv, B, T, L, H, D, wl.scale, wl.topk,
+                                                wl.window, block, dt, O, None, idx, ns, ws, nb,
+                                                stream)
+            else:
+                hs2.hs2_full_attn_select(q, kv, B, T, L, H, D, wl.scale, wl.topk, wl.window, dt,
+                                         O, None, idx, ns, ws, nb, stream)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(10):
+            flush_fn()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        st = hs2.hs2_last_device_status()
+        if st != 0:
+            raise RuntimeError("block selection device status: " + hs2.hs2_status_string(st))
+        gi = idx.cpu().numpy().reshape(B * T, slots)
+        gn = ns.cpu().numpy().reshape(-1)
+        hit = [int(j) in set(gi[b * T + t, :gn[b * T + t]].tolist()) for b, j, t in inp.needles]
+        out[label] = {"full_ms": float(np.median(ts)), "needle_recall": float(np.mean(hit))}
+    out["needles"] = int(len(inp.needles))
+    out["budget"] = "%d positions + %d window" % (wl.topk, wl.window)
+    return out
+
+
 # ------------------------------------------------------- other configurations --
-def bench_other_configs(torch, hs2, stream, flush_fn, peak_gbs, peak_tflops):
+def bench_other_configs(torch, hs2, stream, flush_fn, peak_gbs, peak_tflops,
+                        names=("decode_fp8_256k", "chunk_fp8_1m")):
     """Times the full-attention call and one sparse layer on the E4M3 configurations
     (4 x 256K decode; the 4096-query chunk over a 1M-token cache), beside the decode
     metric.  Inputs are drawn on the device in the workloads' distributions (Q, K, V
@@ -274,6 +380,8 @@ def bench_other_configs(torch, hs2, stream, flush_fn, peak_gbs, peak_tflops):
     every timed call; parity of these shapes is covered by the test suite."""
     out = {}
     for name, reps in (("decode_fp8_256k", 10), ("chunk_fp8_1m", 3)):
+        if name not in names:
+            continue
         wl = WORKLOADS[name]
         B, T, L, H, D = wl.B, wl.T, wl.L, wl.H, wl.D
         g = torch.Generator(device="cuda").manual_seed(wl.seed)
@@ -569,6 +677,10 @@ def run_hs2(args, world, rank, local):
                "sample": "one full step: %d sequences x 1 query, full attention + selection + "
                          "%d sparse layers (%.1f s)" % (B, wl.n_sparse, dts)}
     bridge = bench_bridge(torch, hs2, args, stream) if (rank == 0 and not args.no_bridge) else None
+    append = (bench_bridge_append(torch, hs2, stream, l2_flush, peak)
+              if (rank == 0 and not args.no_bridge) else None)
+    blocks = (bench_block_selection(torch, hs2, inp, kv, qs[0], stream, l2_flush)
+              if rank == 0 and not args.no_configs else None)
     others = None
     if rank == 0 and not args.no_configs:
         others = bench_other_configs(torch, hs2, stream, l2_flush, peak,
@@ -616,15 +728,48 @@ def run_hs2(args, world, rank, local):
         "clocks": clk,
         "cpu_baseline": cpu,
         "bridge": bridge,
+        "bridge_append": append,
+        "block_selection": blocks,
         "configs": others,
     }
     print(json.dumps(line), flush=True)
 
 
+def run_section(args):
+    """One section of the GPU arm alone (no headline step): for profiling."""
+    import torch
+    import long_context_hs2_b200 as hs2
+    torch.cuda.set_device(0)
+    hs2.load_library()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def l2_flush():
+        flush.zero_()
+        flush.view(torch.int64).amax()
+
+    peak, _ = measured_peaks()
+    if args.only == "append":
+        out = bench_bridge_append(torch, hs2, stream, l2_flush, peak)
+    elif args.only == "blocks":
+        inp = make_attention_inputs(WORKLOADS[WORKLOAD])
+        up = (lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+              .view(torch.bfloat16))
+        kv = hs2.kv_cache(up(inp.k), up(inp.v))
+        out = bench_block_selection(torch, hs2, inp, kv, up(inp.q), stream, l2_flush)
+    else:
+        names = ("decode_fp8_256k", "chunk_fp8_1m") if args.only == "configs" else (args.only,)
+        out = bench_other_configs(torch, hs2, stream, l2_flush, peak, measured_tensor_peak()[0],
+                                  names)
+    print(json.dumps({"section": args.only, args.only: out}), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup()
-    if args.impl == "reference":
+    if args.only:
+        run_section(args)
+    elif args.impl == "reference":
         run_reference(args, world, rank)
     else:
         run_hs2(args, world, rank, local)
