@@ -54,11 +54,15 @@ constexpr float kRescaleAbove = 8.f;  // base-2 logits may exceed the reference 
 // histograms.
 template <int N, bool FP8>
 struct TcSmem {
-  static constexpr int kStages = FP8 ? (N == 32 ? 4 : 2) : (N == 32 ? 3 : 2);
+  static constexpr int kStages = N == 32 ? 3 : 2;
   static constexpr int kNP = N == 32 ? 2 : 1;            // P^T buffers
   static constexpr int kStageBytes = 2 * (FP8 ? kTcTile8Bytes : kTcTileBytes);  // K then V
-  static constexpr int kK16Off = kStages * kStageBytes;  // E4M3 only: f16 K, then f16 V
-  static constexpr int kQOff = kK16Off + (FP8 ? 2 * kTcTileBytes : 0);
+  // E4M3 only: converted f16 K tiles (two for 32-row groups, so the converters
+  // write tile n+1 while the tensor cores read tile n), then the f16 V tile
+  static constexpr int kNK16 = (FP8 && N == 32) ? 2 : 1;
+  static constexpr int kK16Off = kStages * kStageBytes;
+  static constexpr int kV16Off = kK16Off + kNK16 * kTcTileBytes;
+  static constexpr int kQOff = kK16Off + (FP8 ? (kNK16 + 1) * kTcTileBytes : 0);
   static constexpr int kQBytes = N * 256;
   static constexpr int kPOff = kQOff + kQBytes;          // P^T [N rows][128 keys], 16-bit
   static constexpr int kPBytes = N * 256;
@@ -66,7 +70,7 @@ struct TcSmem {
   static constexpr int kCorrOff = kMrefOff + N * 4;      // float [N]
   static constexpr int kTmaxOff = kCorrOff + N * 4;      // float [4][N] (also the row sums)
   static constexpr int kBarOff = kTmaxOff + 4 * N * 4;
-  static constexpr int kNumBars = 3 * kStages + 9 + 2 * kNP;  // + V arrival per stage
+  static constexpr int kNumBars = 3 * kStages + 11 + 2 * kNP;  // + V arrival per stage, second f16 K
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBar2Off = kSlotOff + 16;         // fused kernel: score-pass barriers
   static constexpr int kNumBars2 = 16;
@@ -80,8 +84,12 @@ struct TcSmem {
   static constexpr int kS2Stages = 4;
   static constexpr int kS2TileBytes = FP8 ? kTcTile8Bytes : kTcTileBytes;
   static constexpr int kS2MlOff = kS2Stages * kS2TileBytes;  // float2 [N][splits], <= 32 KB
-  static constexpr int kS2HistOff = kS2MlOff + 32 * 1024;    // unsigned [G][2048], <= 32 KB
-  static constexpr bool kFusable = kS2HistOff + 32 * 1024 <= kRingBytes;
+  // unsigned [G][2048], <= 32 KB: in the f16 V tile for E4M3 (idle in the score
+  // pass, whose two f16 K tiles are the partial pass's), else after the (m, l)
+  static constexpr bool kHistInV16 = FP8 && N == 32;
+  static constexpr int kS2HistOff = kHistInV16 ? kV16Off : kS2MlOff + 32 * 1024;
+  static constexpr bool kFusable =
+      (kHistInV16 ? kS2MlOff : kS2HistOff) + 32 * 1024 <= kRingBytes;
   static constexpr int kSelWorkOff = kRingBytes - 16 * 1024;  // counters, list offsets
   static constexpr int kSelCap = kSelWorkOff / 4;             // list entries held in smem
   // score kernel
@@ -254,6 +262,8 @@ __device__ __forceinline__ void tc_partial_setup(uint8_t* smem) {
     mbar_init(q_ready + 3, kTcConvert / 32);  // v16_full
     mbar_init(q_ready + 4, 1);                // v16_free
     for (int s = 0; s < S; ++s) mbar_init(q_ready + 5 + s, 1);  // v_full (bf16: V of stage s)
+    mbar_init(q_ready + 5 + S, kTcConvert / 32);  // k16_full of the second f16 K tile
+    mbar_init(q_ready + 6 + S, 1);                // its k16_free
     fence_mbar_init();
   }
 }
@@ -298,6 +308,11 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
   uint64_t* v16_full = k16_free + 1;
   uint64_t* v16_free = v16_full + 1;
   uint64_t* v_full = v16_free + 1;   // [S] bf16: V of a stage (kv_full then means K)
+  // E4M3: f16 K tile n sits in buffer n % kNK16, with its own full/free pair
+  constexpr int NK = SM::kNK16;
+  auto k16_full_of = [&](int n) { return (NK == 2 && (n & 1)) ? v_full + S : k16_full; };
+  auto k16_free_of = [&](int n) { return (NK == 2 && (n & 1)) ? v_full + S + 1 : k16_free; };
+  auto k16_use = [&](int n) { return (uint32_t)((n / NK) & 1); };   // phase of tile n's use
 
   const int split = blockIdx.x % p.n_splits;
   const int grp = blockIdx.x / p.n_splits;
@@ -353,7 +368,7 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
     // -------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t k16_addr = smem_u32(smem + SM::kK16Off);
-      const uint32_t v16_addr = k16_addr + kTcTileBytes;
+      const uint32_t v16_addr = smem_u32(smem + SM::kV16Off);
       bool ok = true;
       auto pv = [&](int m) {
         if (!mbar_wait(&p_full[m % NP], (m / NP) & 1)) return false;
@@ -370,13 +385,15 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
       ok = mbar_wait(q_ready, 0);  // Q staged by the softmax warps
       for (int n = 0; n < n_tiles && ok; ++n) {
         const int s = n % S, bb = n & 1;
-        if (!mbar_wait(FP8 ? k16_full : &kv_full[s], FP8 ? (n & 1) : (n / S) & 1)) break;
+        if (!mbar_wait(FP8 ? k16_full_of(n) : &kv_full[s], FP8 ? k16_use(n) : (n / S) & 1)) break;
         if (!RETAIN && n >= 2 && !mbar_wait(&s_empty[bb], ((n - 2) >> 1) & 1)) break;
         tc_fence_after();
-        tc_issue_qk<N, FP8>(tmem + s_col(n), FP8 ? k16_addr : smem_u32(smem + s * SM::kStageBytes),
+        tc_issue_qk<N, FP8>(tmem + s_col(n),
+                            FP8 ? k16_addr + (uint32_t)((n % NK) * kTcTileBytes)
+                                : smem_u32(smem + s * SM::kStageBytes),
                             q_addr);
         tc_commit(&s_full[bb]);
-        if (FP8) tc_commit(k16_free);
+        if (FP8) tc_commit(k16_free_of(n));
         if (n >= 1) ok = pv(n - 1);
       }
       if (ok) pv(n_tiles - 1);
@@ -386,13 +403,15 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
     const int ct = threadIdx.x - (64 + kTcSoftmax);  // 0..127
     const bool is_v = ct >= kTcConvert;
     const int cid = ct % kTcConvert;
-    uint8_t* dst = smem + SM::kK16Off + (is_v ? kTcTileBytes : 0);
-    uint64_t* full16 = is_v ? v16_full : k16_full;
-    uint64_t* free16 = is_v ? v16_free : k16_free;
+    const int nbuf = is_v ? 1 : NK;   // f16 buffers of this tensor
     for (int n = 0; n < n_tiles; ++n) {
       const int s = n % S;
+      uint8_t* dst = smem + (is_v ? SM::kV16Off : SM::kK16Off + (n % nbuf) * kTcTileBytes);
+      uint64_t* full16 = is_v ? v16_full : k16_full_of(n);
+      uint64_t* free16 = is_v ? v16_free : k16_free_of(n);
       if (!mbar_wait(&kv_full[s], (n / S) & 1)) break;
-      if (n >= 1 && !mbar_wait(free16, (n - 1) & 1)) break;  // MMA done with the last tile
+      // the MMAs are done with the tile this buffer held before (tile n - nbuf)
+      if (n >= nbuf && !mbar_wait(free16, ((n - nbuf) / nbuf) & 1)) break;
       fp8_rows_to_f16(smem + s * SM::kStageBytes + (is_v ? kTileIn : 0), 0, kTcKeys, cid,
                       kTcConvert, dst);
       fence_proxy_async_smem();
@@ -842,9 +861,21 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     // warps 2-9: the group's (m, l) partials and lse (base 2) of its rows
     const int st = threadIdx.x - 64;
     const float2* ml_g = p.part_ml + (long long)grp * ns * N;
-    for (int u = st; u < N * ns; u += kTcSoftmax) {
-      const int sp = u / N, r = u % N;
-      ml_s[r * ns + sp] = __ldcg(ml_g + (long long)sp * N + r);
+    {
+      constexpr int kLoadBatch = 4;   // independent L2 loads in flight per thread
+      for (int u0 = st; u0 < N * ns; u0 += kLoadBatch * kTcSoftmax) {
+        float2 v[kLoadBatch];
+#pragma unroll
+        for (int k = 0; k < kLoadBatch; ++k) {
+          const int u = u0 + k * kTcSoftmax;
+          v[k] = u < N * ns ? __ldcg(ml_g + u) : make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < kLoadBatch; ++k) {
+          const int u = u0 + k * kTcSoftmax;
+          if (u < N * ns) ml_s[(u % N) * ns + u / N] = v[k];
+        }
+      }
     }
     softmax_sync<kTcSoftmax>();
     for (int r = st; r < N; r += kTcSoftmax) {
@@ -917,9 +948,9 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         for (int q = 0; q < G; ++q) {
           const int t = t0 + q;
           const bool cand = t < p.T && j <= p.qpos0 + t - p.window;
-          if (cand) {
-            p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
+          if (cand) {  // the fused selection reads the shared-memory copy only
             if (p.fuse_select) seg[q * p.split_keys + (int)(j - k_lo)] = acc[q];
+            else p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
           }
           hist_inc(hist_s + q * kHistBins, __float_as_uint(acc[q]) >> kHistShift, cand);
         }
@@ -946,11 +977,19 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         }
         const float* po = p.part_o + ((long long)grp * ns * N + r) * 128 + d;
         float acc = 0.f;
-#pragma unroll 8
-        for (int sp = 0; sp < ns; ++sp) {
-          const float2 v = ml_s[r * ns + sp];
-          const float f = (v.x == kNegInf) ? 0.f : fast_exp2(v.x - l2);
-          acc += f * __ldcg(po + (long long)sp * N * 128);
+        constexpr int kLoadBatch = 16;   // the splits' values of element d, loaded together
+        for (int sp0 = 0; sp0 < ns; sp0 += kLoadBatch) {
+          float x[kLoadBatch];
+#pragma unroll
+          for (int k = 0; k < kLoadBatch; ++k)
+            x[k] = sp0 + k < ns ? __ldcg(po + (long long)(sp0 + k) * N * 128) : 0.f;
+#pragma unroll
+          for (int k = 0; k < kLoadBatch; ++k) {
+            if (sp0 + k >= ns) break;
+            const float2 v = ml_s[r * ns + sp0 + k];
+            const float f = (v.x == kNegInf) ? 0.f : fast_exp2(v.x - l2);
+            acc += f * x[k];
+          }
         }
         p.o[li * 128 + d] = acc;
       }
@@ -1063,26 +1102,48 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
           }
           return __ldcg(list_g(q, lo) + (e - off_s[lo]));
         };
-        if (in_smem)
-          for (int e = threadIdx.x; e < m; e += kThreads) list_s[e] = list_at(e);
-        __syncthreads();
-        auto val = [&](int e) { return in_smem ? list_s[e] : list_at(e); };
-        // level 2: bits [19:9] of the list (every element is in b1)
-        for (int e = threadIdx.x; e < m; e += kThreads) hist_inc(h, (val(e) >> 9) & 2047u, true);
-        __syncthreads();
-        sel_find_bin<kThreads>(h, 2048, s_need[q], s_res, s_tmp);
-        const unsigned pre2 = ((unsigned)s_prefix[q] << 11) | (unsigned)s_res[0];
-        const int need2 = s_res[1];
-        for (int e = threadIdx.x; e < 512; e += kThreads) h[e] = 0u;
-        __syncthreads();
-        for (int e = threadIdx.x; e < m; e += kThreads) {
-          const unsigned v = val(e);
-          hist_inc(h, v & 511u, (v >> 9) == pre2);
+        if (in_smem) {
+          // kLoadBatch independent L2 loads in flight per thread (the list can
+          // hold thousands of entries: one round trip per entry would dominate)
+          constexpr int kLoadBatch = 8;
+          for (int e0 = threadIdx.x; e0 < m; e0 += kLoadBatch * kThreads) {
+            unsigned v[kLoadBatch];
+#pragma unroll
+            for (int u = 0; u < kLoadBatch; ++u) {
+              const int e = e0 + u * kThreads;
+              v[u] = e < m ? list_at(e) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kLoadBatch; ++u) {
+              const int e = e0 + u * kThreads;
+              if (e < m) list_s[e] = v[u];
+            }
+          }
         }
         __syncthreads();
-        sel_find_bin<kThreads>(h, 512, need2, s_res, s_tmp);
-        const unsigned tau = (pre2 << 9) | (unsigned)s_res[0];
-        const int need_tau = s_res[1];
+        auto val = [&](int e) { return in_smem ? list_s[e] : list_at(e); };
+        // levels 2 and 3 -- bits [19:9], then [8:0], of the list's elements that
+        // share the digits found so far -- as one loop over the same code (it
+        // runs once per launch, so every distinct instruction is fetched cold)
+        unsigned tau = (unsigned)s_prefix[q];
+        int need_tau = s_need[q];
+#pragma unroll 1
+        for (int lvl = 0; lvl < 2; ++lvl) {
+          const int shift = lvl == 0 ? 9 : 0, nbins = lvl == 0 ? 2048 : 512;
+          const int kept = lvl == 0 ? 20 : 9;   // bits above the digit: those found so far
+          if (lvl == 1) {
+            for (int e = threadIdx.x; e < 512; e += kThreads) h[e] = 0u;
+            __syncthreads();
+          }
+          for (int e = threadIdx.x; e < m; e += kThreads) {
+            const unsigned v = val(e);
+            hist_inc(h, (v >> shift) & (unsigned)(nbins - 1), (v >> kept) == tau);
+          }
+          __syncthreads();
+          sel_find_bin<kThreads>(h, nbins, need_tau, s_res, s_tmp);
+          tau = (tau << (lvl == 0 ? 11 : 9)) | (unsigned)s_res[0];
+          need_tau = s_res[1];
+        }
         // survivors of the lower splits' b1 slices: above tau, and ties
         const int own = s_base[1];
         int a = 0, tie = 0;

@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <utility>
 
@@ -364,16 +365,62 @@ hs2_status run_select_blocks(const FullAttnParams& fp, int topk, int window, int
                 bytes, s, 1, bp);
 }
 
+// Shared memory of a sparse launch: the position array holds one CTA's share
+// of the slots in whole tiles, plus n_sel.
 template <int MT, int D, bool FP8>
-hs2_status run_sparse(const SparseParams& p, cudaStream_t s) {
+size_t sparse_smem_bytes(int slots, int cs) {
+  const int tiles_max = (sparse_share(slots, cs) + kSpTile - 1) / kSpTile;
+  return (size_t)SparseSmem<MT, D, FP8>::kPosOff + (size_t)(tiles_max * kSpTile + 4) * 4 + 1024;
+}
+
+// p.cs is the power-of-two cluster size chosen by the caller.  When the
+// slots of a query fill ceil(slots / tile) CTAs of one tile each and clusters
+// of that size (up to 16, a non-portable size) are co-resident for every
+// query at once, that size is used instead: each CTA then has a single tile.
+template <int MT, int D, bool FP8>
+hs2_status run_sparse(SparseParams p, cudaStream_t s) {
   using SM = SparseSmem<MT, D, FP8>;
   auto k = sparse_attn_kernel<MT, D, FP8>;
   if (!set_smem(k, SM::kBytes)) return HS2_ERR_CUDA;
-  // the position array holds one CTA's share of the slots in whole tiles, plus n_sel
-  const int tiles_max = (sparse_share(p.slots, p.cs) + kSpTile - 1) / kSpTile;
-  const size_t bytes = (size_t)SM::kPosOff + (size_t)(tiles_max * kSpTile + 4) * 4 + 1024;
-  return launch_ex(k, dim3((unsigned)((long long)p.B * p.T * p.cs)), dim3(kSpThreads), bytes, s,
-                   p.cs, false, true, p);
+  const long long queries = (long long)p.B * p.T;
+  const int want = (p.slots + kSpTile - 1) / kSpTile;
+  // co-resident clusters of `want` CTAs, per device and slot count (queried once)
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, int> resident;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int n_res = -1;
+  if (want > p.cs && want <= 16 && queries * want <= sm_count()) {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = resident.find({dev, p.slots});
+    if (it != resident.end()) n_res = it->second;
+  }
+  if (n_res < 0 && want > p.cs && want <= 16 && queries * want <= sm_count()) {
+    n_res = 0;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(queries * want));
+      cfg.blockDim = dim3(kSpThreads);
+      cfg.dynamicSmemBytes = sparse_smem_bytes<MT, D, FP8>(p.slots, want);
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = (unsigned)want;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int n_clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&n_clusters, k, &cfg) == cudaSuccess) n_res = n_clusters;
+    }
+    cudaGetLastError();
+    std::lock_guard<std::mutex> lock(mu);
+    resident[{dev, p.slots}] = n_res;
+  }
+  if (n_res >= queries) p.cs = want;
+  const size_t bytes = sparse_smem_bytes<MT, D, FP8>(p.slots, p.cs);
+  return launch_ex(k, dim3((unsigned)(queries * p.cs)), dim3(kSpThreads), bytes, s, p.cs, false,
+                   true, p);
 }
 
 }  // namespace

@@ -58,7 +58,9 @@ struct SparseSmem {
   static constexpr int kQOff = kMain;
   static constexpr int kMlOff = kQOff + kRowsQ * D * 2;
   static constexpr int kClOff = kMlOff + kSpWarps * kRowsQ * 8;  // merge inputs
-  static constexpr int kClBytes = kRowsQ * 8 + kRowsQ * D * 4;
+  // cs * ceil(H / cs) rows: at most H + cs - 1 for clusters of up to 16 CTAs
+  static constexpr int kClRows = kRowsQ + 16;
+  static constexpr int kClBytes = kClRows * 8 + kClRows * D * 4;
   static constexpr int kPosOff = kClOff + kClBytes;               // positions of the CTA's slots
   static constexpr int kMaxSlots = 4096;
   static constexpr int kBytes = kPosOff + (kMaxSlots + kSpTile + 4) * 4 + 1024;
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(kSpThreads) sparse_attn_kernel(const SparsePar
   // merge inputs: with a cluster, [source CTA][row of this CTA's slice] (m, l)
   // and [source CTA][element of the slice] O, written by the cluster's CTAs
   float2* cl_ml = reinterpret_cast<float2*>(smem + SM::kClOff);
-  float* cl_o = reinterpret_cast<float*>(smem + SM::kClOff + SM::kRowsQ * 8);
+  float* cl_o = reinterpret_cast<float*>(smem + SM::kClOff + SM::kClRows * 8);
   int* pos_all = reinterpret_cast<int*>(smem + SM::kPosOff);  // [tiles][kSpTile]
 
   const int cs = p.cs;
@@ -270,9 +272,11 @@ __global__ void __launch_bounds__(kSpThreads) sparse_attn_kernel(const SparsePar
   float* obuf = reinterpret_cast<float*>(smem);
   warp_store_o<MT, D>(st, f, obuf + warp * SM::kRowsQ * (D + 8));
   // CTA `rank` of the cluster owns rows [rank*rpc, (rank+1)*rpc) of the H x D
-  // output (H / cs is a whole number: H in {8, 16, 32}, cs in {1, 2, 4, 8})
-  const int rpc = p.H / cs;
+  // output, rpc = ceil(H / cs): the last owner may own fewer rows, and CTAs past
+  // it none (cs need not divide H)
+  const int rpc = (p.H + cs - 1) / cs;
   const int chunk = rpc * D;
+  const int own_rows = max(0, min(rpc, p.H - (int)rank * rpc));
   const uint32_t ml_addr = smem_u32(cl_ml), o_addr = smem_u32(cl_o);
   if (cs > 1) cluster_wait_acquire();  // first phase: every CTA of the cluster runs
   __syncthreads();
@@ -326,7 +330,7 @@ __global__ void __launch_bounds__(kSpThreads) sparse_attn_kernel(const SparsePar
   // shared memory after it, so each CTA may exit when its slice is written
   cluster_arrive_release();
   cluster_wait_acquire();
-  for (int e = 4 * threadIdx.x; e < chunk; e += 4 * kSpThreads) {
+  for (int e = 4 * threadIdx.x; e < own_rows * D; e += 4 * kSpThreads) {
     const int rl = e / D;
     float M = kNegInf;
     for (int q = 0; q < cs; ++q) M = fmaxf(M, cl_ml[q * rpc + rl].x);
