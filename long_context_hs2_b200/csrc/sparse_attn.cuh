@@ -49,7 +49,10 @@ struct SparseSmem {
   static constexpr int kRowsQ = MT * 16;
   static constexpr int kElem = FP8 ? 1 : 2;
   static constexpr int kTileBytes = kSpTile * D * kElem;
-  static constexpr int kStages = 2;
+  // ring stages: a query with many tiles (one CTA per query) keeps kStages - 1
+  // tiles of gathers in flight; E4M3 tiles are half the size, so three fit
+  // beside the per-warp f16 staging
+  static constexpr int kStages = FP8 ? 3 : 2;
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kStagingBytes = FP8 ? kSpWarps * 2 * kSpGroup * D * 2 : 0;
   static constexpr int kObufBytes = kSpWarps * kRowsQ * (D + 8) * 4;
@@ -64,6 +67,7 @@ struct SparseSmem {
   static constexpr int kPosOff = kClOff + kClBytes;               // positions of the CTA's slots
   static constexpr int kMaxSlots = 4096;
   static constexpr int kBytes = kPosOff + (kMaxSlots + kSpTile + 4) * 4 + 1024;
+  static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
 // 4-byte global->shared copy (the L1-allocating form; the .cg form moves 16
