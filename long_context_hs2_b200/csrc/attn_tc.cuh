@@ -47,51 +47,57 @@ constexpr int kTcTileBytes = kTcKeys * 128 * 2;   // one 16-bit K or V tile: 32 
 constexpr int kTcTile8Bytes = kTcKeys * 128;      // one E4M3 K or V tile: 16 KB
 constexpr float kRescaleAbove = 8.f;  // base-2 logits may exceed the reference by this
 
-// Shared-memory plan.  Partial kernel: K/V tile ring (16-bit, or E4M3 plus one
-// f16 K and one f16 V tile), Q, P^T (double-buffered for N = 32), per-row
-// reference max / correction / partial maxima and sums.  Score kernel: K ring
-// (plus two f16 K tiles for E4M3), staged (m, l) partials of the group, Q,
-// histograms.
+// Shared-memory plan.  Partial kernel: K/V tile ring (16-bit, or E4M3 plus
+// f16 K and V tiles), Q, P^T (double-buffered for N = 32), per-row reference
+// max / correction / partial maxima and sums.  Score kernel: K ring (plus two
+// f16 K tiles for E4M3), staged (m, l) partials of the group, Q, histograms.
 template <int N, bool FP8>
 struct TcSmem {
-  static constexpr int kStages = N == 32 ? 3 : 2;
+  // E4M3 32-row groups: a 2-stage E4M3 ring (the f16 tiles buffer two more)
+  static constexpr int kStages = N == 32 ? (FP8 ? 2 : 3) : 2;
   static constexpr int kNP = N == 32 ? 2 : 1;            // P^T buffers
   static constexpr int kStageBytes = 2 * (FP8 ? kTcTile8Bytes : kTcTileBytes);  // K then V
-  // E4M3 only: converted f16 K tiles (two for 32-row groups, so the converters
-  // write tile n+1 while the tensor cores read tile n), then the f16 V tile
+  // E4M3 only: converted f16 K tiles, then f16 V tiles -- two of each for
+  // 32-row groups, so the converters write tile n+1 while the tensor cores
+  // read tile n
   static constexpr int kNK16 = (FP8 && N == 32) ? 2 : 1;
+  static constexpr int kNV16 = (FP8 && N == 32) ? 2 : 1;
   static constexpr int kK16Off = kStages * kStageBytes;
   static constexpr int kV16Off = kK16Off + kNK16 * kTcTileBytes;
-  static constexpr int kQOff = kK16Off + (FP8 ? (kNK16 + 1) * kTcTileBytes : 0);
+  static constexpr int kQOff = kK16Off + (FP8 ? (kNK16 + kNV16) * kTcTileBytes : 0);
   static constexpr int kQBytes = N * 256;
-  static constexpr int kPOff = kQOff + kQBytes;          // P^T [N rows][128 keys], 16-bit
+  static constexpr int kPOff = kQOff + kQBytes;  // P^T [N rows][128 keys] (N = 128: P MN-major), 16-bit
   static constexpr int kPBytes = N * 256;
   static constexpr int kMrefOff = kPOff + kNP * kPBytes; // float [N]
   static constexpr int kCorrOff = kMrefOff + N * 4;      // float [N]
   static constexpr int kTmaxOff = kCorrOff + N * 4;      // float [4][N] (also the row sums)
   static constexpr int kBarOff = kTmaxOff + 4 * N * 4;
-  static constexpr int kNumBars = 3 * kStages + 11 + 2 * kNP;  // + V arrival per stage, second f16 K
+  // + V arrival per stage, second f16 K and V tiles
+  static constexpr int kNumBars = 3 * kStages + 13 + 2 * kNP;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBar2Off = kSlotOff + 16;         // fused kernel: score-pass barriers
-  static constexpr int kNumBars2 = 16;
-  static constexpr int kMhistOff = kBar2Off + kNumBars2 * 8;  // retained tiles' references
+  static constexpr int kNumBars2 = 17;  // + the row copy of the fused selection
+  // retained tiles' references (16-byte aligned: read as float4)
+  static constexpr int kMhistOff = (kBar2Off + kNumBars2 * 8 + 15) / 16 * 16;
   static constexpr int kMhistBytes = N == 32 ? 15 * N * 4 : 0;
   static constexpr int kBytes = kMhistOff + kMhistBytes + 1024;
   // fused kernel: the score pass reuses the partial pass's tile ring for its
-  // K ring, the group's (m, l) partials and the histograms; the fused
-  // selection then uses it for the row's candidate scores and its counters
+  // K ring, the group's (m, l) partials float2 [N][splits] and the
+  // histograms unsigned [G][2048] (<= 32 KB each): after the K ring, or for
+  // E4M3 in the two f16 V tiles (idle in the score pass, whose two f16 K tiles
+  // are the partial pass's).  The fused selection then uses everything below Q
+  // for the row's candidate scores and its counters.
   static constexpr int kRingBytes = kStages * kStageBytes;
   static constexpr int kS2Stages = 4;
   static constexpr int kS2TileBytes = FP8 ? kTcTile8Bytes : kTcTileBytes;
-  static constexpr int kS2MlOff = kS2Stages * kS2TileBytes;  // float2 [N][splits], <= 32 KB
-  // unsigned [G][2048], <= 32 KB: in the f16 V tile for E4M3 (idle in the score
-  // pass, whose two f16 K tiles are the partial pass's), else after the (m, l)
   static constexpr bool kHistInV16 = FP8 && N == 32;
+  static constexpr int kS2MlOff = kHistInV16 ? kV16Off + 32 * 1024 : kS2Stages * kS2TileBytes;
   static constexpr int kS2HistOff = kHistInV16 ? kV16Off : kS2MlOff + 32 * 1024;
   static constexpr bool kFusable =
-      (kHistInV16 ? kS2MlOff : kS2HistOff) + 32 * 1024 <= kRingBytes;
-  static constexpr int kSelWorkOff = kRingBytes - 16 * 1024;  // counters, list offsets
-  static constexpr int kSelCap = kSelWorkOff / 4;             // list entries held in smem
+      kHistInV16 ? (kS2Stages * kS2TileBytes <= kRingBytes && kNV16 * kTcTileBytes >= 64 * 1024)
+                 : kS2HistOff + 32 * 1024 <= kRingBytes;
+  static constexpr int kSelWorkOff = kQOff - 16 * 1024;  // counters, list offsets
+  static constexpr int kSelCap = kSelWorkOff / 4;        // list entries held in smem
   // score kernel
   static constexpr int kSStages = (FP8 || N == 32) ? 4 : 3;
   static constexpr int kSStageBytes = FP8 ? kTcTile8Bytes : kTcTileBytes;
@@ -199,18 +205,26 @@ __device__ __forceinline__ void tc_issue_qk(uint32_t tmem_d, uint32_t k_addr, ui
   }
 }
 
+// P operand layout of the PV product: 128-row groups store P MN-major (each
+// key's rows contiguous, so a softmax thread writes 16-byte chunks), 32-row
+// groups P^T K-major (a key's 16 rows would fill only a quarter of a row).
+__host__ __device__ constexpr bool tc_p_mn_major(int N) { return N == 128; }
+
 // Issues the 8 MMAs of O^T[128 x N] (+)= V_tile^T . P, V read MN-major from its
-// TMA tile (d contiguous within a 64-d half, halves 16 KB apart), P^T K-major.
+// TMA tile (d contiguous within a 64-d half, halves 16 KB apart); P MN-major
+// in the same geometry (64-row halves 16 KB apart) or P^T K-major.
 template <int N, bool F16>
 __device__ __forceinline__ void tc_issue_pv(uint32_t tmem_d, uint32_t v_addr, uint32_t p_addr,
                                             bool accumulate) {
-  constexpr uint32_t idesc = tc_idesc_f16(128, N, F16 ? kTcF16 : kTcBF16, true, false);
+  constexpr bool kPMN = tc_p_mn_major(N);
+  constexpr uint32_t idesc = tc_idesc_f16(128, N, F16 ? kTcF16 : kTcBF16, true, kPMN);
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
     const uint32_t half = ks >> 2, koff = (ks & 3) * 32;
     tc_mma_f16(tmem_d, sw128_mnmajor_desc(v_addr + ks * 16 * 128, kTcKeys * 128),
-               sw128_kmajor_desc(p_addr + half * (N * 128) + koff), idesc,
-               accumulate || ks > 0);
+               kPMN ? sw128_mnmajor_desc(p_addr + ks * 16 * 128, kTcKeys * 128)
+                    : sw128_kmajor_desc(p_addr + half * (N * 128) + koff),
+               idesc, accumulate || ks > 0);
   }
 }
 
@@ -264,6 +278,8 @@ __device__ __forceinline__ void tc_partial_setup(uint8_t* smem) {
     for (int s = 0; s < S; ++s) mbar_init(q_ready + 5 + s, 1);  // v_full (bf16: V of stage s)
     mbar_init(q_ready + 5 + S, kTcConvert / 32);  // k16_full of the second f16 K tile
     mbar_init(q_ready + 6 + S, 1);                // its k16_free
+    mbar_init(q_ready + 7 + S, kTcConvert / 32);  // v16_full of the second f16 V tile
+    mbar_init(q_ready + 8 + S, 1);                // its v16_free
     fence_mbar_init();
   }
 }
@@ -308,11 +324,16 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
   uint64_t* v16_full = k16_free + 1;
   uint64_t* v16_free = v16_full + 1;
   uint64_t* v_full = v16_free + 1;   // [S] bf16: V of a stage (kv_full then means K)
-  // E4M3: f16 K tile n sits in buffer n % kNK16, with its own full/free pair
+  // E4M3: f16 K tile n sits in buffer n % kNK16, V tile n in buffer n % kNV16,
+  // each buffer with its own full/free pair
   constexpr int NK = SM::kNK16;
+  constexpr int NV = SM::kNV16;
   auto k16_full_of = [&](int n) { return (NK == 2 && (n & 1)) ? v_full + S : k16_full; };
   auto k16_free_of = [&](int n) { return (NK == 2 && (n & 1)) ? v_full + S + 1 : k16_free; };
   auto k16_use = [&](int n) { return (uint32_t)((n / NK) & 1); };   // phase of tile n's use
+  auto v16_full_of = [&](int n) { return (NV == 2 && (n & 1)) ? v_full + S + 2 : v16_full; };
+  auto v16_free_of = [&](int n) { return (NV == 2 && (n & 1)) ? v_full + S + 3 : v16_free; };
+  auto v16_use = [&](int n) { return (uint32_t)((n / NV) & 1); };
 
   const int split = blockIdx.x % p.n_splits;
   const int grp = blockIdx.x / p.n_splits;
@@ -372,14 +393,15 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
       bool ok = true;
       auto pv = [&](int m) {
         if (!mbar_wait(&p_full[m % NP], (m / NP) & 1)) return false;
-        if (FP8 && !mbar_wait(v16_full, m & 1)) return false;
+        if (FP8 && !mbar_wait(v16_full_of(m), v16_use(m))) return false;
         if (!FP8 && !mbar_wait(&v_full[m % S], (m / S) & 1)) return false;
         tc_fence_after();
         tc_issue_pv<N, FP8>(tmem + kOCol,
-                            FP8 ? v16_addr : smem_u32(smem + (m % S) * SM::kStageBytes + kTileIn),
+                            FP8 ? v16_addr + (uint32_t)((m % NV) * kTcTileBytes)
+                                : smem_u32(smem + (m % S) * SM::kStageBytes + kTileIn),
                             p_addr + (m % NP) * SM::kPBytes, m > 0);
         tc_commit(&pv_done[m % NP]);
-        tc_commit(FP8 ? v16_free : &kv_empty[m % S]);
+        tc_commit(FP8 ? v16_free_of(m) : &kv_empty[m % S]);
         return true;
       };
       ok = mbar_wait(q_ready, 0);  // Q staged by the softmax warps
@@ -403,12 +425,12 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
     const int ct = threadIdx.x - (64 + kTcSoftmax);  // 0..127
     const bool is_v = ct >= kTcConvert;
     const int cid = ct % kTcConvert;
-    const int nbuf = is_v ? 1 : NK;   // f16 buffers of this tensor
+    const int nbuf = is_v ? NV : NK;   // f16 buffers of this tensor
     for (int n = 0; n < n_tiles; ++n) {
       const int s = n % S;
-      uint8_t* dst = smem + (is_v ? SM::kV16Off : SM::kK16Off + (n % nbuf) * kTcTileBytes);
-      uint64_t* full16 = is_v ? v16_full : k16_full_of(n);
-      uint64_t* free16 = is_v ? v16_free : k16_free_of(n);
+      uint8_t* dst = smem + (is_v ? SM::kV16Off : SM::kK16Off) + (n % nbuf) * kTcTileBytes;
+      uint64_t* full16 = is_v ? v16_full_of(n) : k16_full_of(n);
+      uint64_t* free16 = is_v ? v16_free_of(n) : k16_free_of(n);
       if (!mbar_wait(&kv_full[s], (n / S) & 1)) break;
       // the MMAs are done with the tile this buffer held before (tile n - nbuf)
       if (n >= nbuf && !mbar_wait(free16, ((n - nbuf) / nbuf) & 1)) break;
@@ -439,7 +461,11 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const int keyrow = wq * 32 + lane;       // row of S^T (key) / of O^T (d)
     // P^T store address of (row c0 + c, this key): base + c*128 + xoff[(c0 + c) & 7]
+    // (K-major P^T); for 128-row groups P is stored MN-major instead: this
+    // key's 128-byte row of the 64-row half c0/64, 16-byte chunks swizzled by key
+    constexpr bool kPMN = tc_p_mn_major(N);
     uint8_t* p_base = smem + SM::kPOff + (keyrow >> 6) * (N * 128) + c0 * 128;
+    uint8_t* pmn_row = smem + SM::kPOff + (c0 / 64) * (kTcKeys * 128) + keyrow * 128;
     uint32_t xoff[8];
 #pragma unroll
     for (int m = 0; m < 8; ++m) xoff[m] = ((((keyrow & 63) >> 3) ^ m) << 4) + (keyrow & 7) * 2;
@@ -479,10 +505,14 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
       tc_fence_after();
       // a tile is "full" when every key is in range and causal for every query
       const bool full_tile = key0 + kTcKeys <= k_hi && key0 + kTcKeys - 1 <= p.qpos0 + t0;
-      // limit[q]: last key query q of the group may see (in range of this split)
-      long long limit[G];
+      // key j (in range) is seen by the group's queries q >= j - qpos0 - t0.  This
+      // thread's columns c0 .. c0+NC-1 are rows of queries c0/kH + (0 .. NQ-1):
+      // vis[(c + i) / kH] is indexed at compile time (a per-query array with a
+      // runtime index would sit in local memory)
+      constexpr int NQ = (NC + kH - 1) / kH;
+      bool vis[NQ];
 #pragma unroll
-      for (int q = 0; q < G; ++q) limit[q] = min(k_hi - 1, p.qpos0 + t0 + q);
+      for (int k = 0; k < NQ; ++k) vis[k] = j < k_hi && (long long)(c0 / kH + k) >= j - p.qpos0 - t0;
       const uint32_t s_addr = tmem + lane_base + s_col(n) + c0;
       // kHold (NC <= 16): this key's logits of the warp's rows are loaded once and
       // kept for both sweeps; wider rows reload 16 columns at a time (registers)
@@ -503,7 +533,7 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
         }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const bool ok = full_tile || j <= limit[(c + i) / kH + c0 / kH];
+          const bool ok = full_tile || vis[(c + i) / kH];
           need |= ok && xs[(kHold ? c : 0) + i] * sl > m_ref[c0 + c + i] + kRescaleAbove;
         }
       }
@@ -523,7 +553,7 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
           }
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const bool ok = full_tile || j <= limit[(c + i) / kH + c0 / kH];
+            const bool ok = full_tile || vis[(c + i) / kH];
             const float v = warp_max(ok ? xs[(kHold ? c : 0) + i] * sl : kNegInf);
             if (lane == 0) tmax[wq * N + c0 + c + i] = v;
           }
@@ -585,17 +615,30 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int col = c0 + c + i;
-          const bool ok = full_tile || j <= limit[(c + i) / kH + c0 / kH];
+          const bool ok = full_tile || vis[(c + i) / kH];
           const float mr = m_ref[col];
           const float pr = (ok && mr != kNegInf) ? fast_exp2(x[i] * sl - mr) : 0.f;
           pk[i] = pr;
           lv[i] += pr;
+          if (kPMN) continue;
           if (FP8)
             *reinterpret_cast<__half*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
                 __float2half_rn(pr * vsc);
           else
             *reinterpret_cast<__nv_bfloat16*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
                 __float2bfloat16_rn(pr);
+        }
+        if (kPMN) {  // this key's 16 rows c0+c .. c0+c+15: two packed 16-byte chunks
+          uint32_t w[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) w[u] = FP8 ? pack_f16(pk[2 * u] * vsc, pk[2 * u + 1] * vsc)
+                                                 : pack_bf16(pk[2 * u], pk[2 * u + 1]);
+          uint8_t* prow = pmn_row + (n % NP) * SM::kPBytes;
+          const int ch = c >> 3;
+          *reinterpret_cast<uint4*>(prow + ((ch ^ (keyrow & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(prow + (((ch + 1) ^ (keyrow & 7)) << 4)) =
+              make_uint4(w[4], w[5], w[6], w[7]);
         }
         if (RETAIN) {
 #pragma unroll
@@ -756,6 +799,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       mbar_init(&k2_full[i], 4);
       mbar_init(&k2_free[i], 1);
     }
+    mbar_init(k2_free + 2, 1);  // the fused selection's row copy
     fence_mbar_init();
   }
   if (threadIdx.x / 32 == 1) {
@@ -861,6 +905,15 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     // warps 2-9: the group's (m, l) partials and lse (base 2) of its rows
     const int st = threadIdx.x - 64;
     const float2* ml_g = p.part_ml + (long long)grp * ns * N;
+    // merge warps 6-9: the partial O of the first row this CTA merges (row
+    // `split`, up to kPre splits) does not depend on lse -- load it now
+    constexpr int kPre = FP8 ? 16 : 32;  // (E4M3: 128 registers per thread)
+    float pre[kPre];
+    if (warp >= 6 && split < N && t0 + split / kH < p.T) {
+      const float* po = p.part_o + ((long long)grp * ns * N + split) * 128 + (threadIdx.x - 192);
+#pragma unroll
+      for (int k = 0; k < kPre; ++k) pre[k] = k < ns ? __ldcg(po + (long long)k * N * 128) : 0.f;
+    }
     {
       constexpr int kLoadBatch = 4;   // independent L2 loads in flight per thread
       for (int u0 = st; u0 < N * ns; u0 += kLoadBatch * kTcSoftmax) {
@@ -912,47 +965,86 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         const long long jn = k_lo + (long long)n * kTcKeys + keyrow;
         return (FP8 && !RETAIN && n < n2 && jn < k2_hi) ? p.k_scale[(long long)b * p.L + jn] : 0.f;
       };
-      float ks_next = load_ks(0);  // E4M3: one tile ahead of its use
-      for (int n = 0; n < n2; ++n) {
-        const int bb = n & 1;
+      // tile n's candidate scores of this key: the selection's copies and histogram
+      auto emit = [&](int n, const float* acc) {
         const long long j = k_lo + (long long)n * kTcKeys + keyrow;
-        float sl = p.scale_log2;
-        if (FP8 && !RETAIN) {
-          sl *= ks_next;
-          ks_next = load_ks(n + 1);
-        }
-        if (!RETAIN && !mbar_wait(&s2_full[bb], (n >> 1) & 1)) break;
-        tc_fence_after();
-        const uint32_t s_col = RETAIN ? N + n * N : bb * N;
-        float acc[G];
-#pragma unroll
-        for (int q = 0; q < G; ++q) acc[q] = 0.f;
-#pragma unroll
-        for (int c = 0; c < N / 32; ++c) {
-          float x[32];
-          tmem_ld32(tmem + lane_base + s_col + 32 * c, x);
-          tmem_ld_wait();
-          if (RETAIN) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc[(32 * c + i) / kH] += x[i] * fct[n * N + 32 * c + i];
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              acc[(32 * c + i) / kH] += fast_exp2(x[i] * sl - lse2_s[32 * c + i]);
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (!RETAIN && lane == 0) mbar_arrive(&s2_empty[bb]);
 #pragma unroll
         for (int q = 0; q < G; ++q) {
           const int t = t0 + q;
           const bool cand = t < p.T && j <= p.qpos0 + t - p.window;
-          if (cand) {  // the fused selection reads the shared-memory copy only
-            if (p.fuse_select) seg[q * p.split_keys + (int)(j - k_lo)] = acc[q];
-            else p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
+          if (cand) {  // the fused selection reads the shared-memory copy (and the row copy)
+            if (p.fuse_select) {
+              seg[q * p.split_keys + (int)(j - k_lo)] = acc[q];
+              if (p.sel_rowscan)
+                p.sel_list[((long long)b * p.T + t) * ns * p.split_keys + j] =
+                    __float_as_uint(acc[q]);
+            } else {
+              p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
+            }
           }
           hist_inc(hist_s + q * kHistBins, __float_as_uint(acc[q]) >> kHistShift, cand);
+        }
+      };
+      if (RETAIN) {
+        // two tiles' blocks per TMEM round trip; each query's 32/G-term dot
+        // product in four independent partial sums
+        auto dot = [&](int n, const float* x, float* acc) {
+          const float4* f4 = reinterpret_cast<const float4*>(fct + n * N);
+          float a4[G][4];
+#pragma unroll
+          for (int q = 0; q < G; ++q) a4[q][0] = a4[q][1] = a4[q][2] = a4[q][3] = 0.f;
+#pragma unroll
+          for (int i4 = 0; i4 < N / 4; ++i4) {
+            const float4 f = f4[i4];
+            const int q = 4 * i4 / kH;
+            a4[q][0] = fmaf(x[4 * i4], f.x, a4[q][0]);
+            a4[q][1] = fmaf(x[4 * i4 + 1], f.y, a4[q][1]);
+            a4[q][2] = fmaf(x[4 * i4 + 2], f.z, a4[q][2]);
+            a4[q][3] = fmaf(x[4 * i4 + 3], f.w, a4[q][3]);
+          }
+#pragma unroll
+          for (int q = 0; q < G; ++q) acc[q] = (a4[q][0] + a4[q][1]) + (a4[q][2] + a4[q][3]);
+        };
+        for (int n = 0; n < n2; n += 2) {
+          float x0[32], x1[32], acc[G];
+          tmem_ld32(tmem + lane_base + N + n * N, x0);
+          if (n + 1 < n2) tmem_ld32(tmem + lane_base + N + (n + 1) * N, x1);
+          tmem_ld_wait();
+          dot(n, x0, acc);
+          emit(n, acc);
+          if (n + 1 < n2) {
+            dot(n + 1, x1, acc);
+            emit(n + 1, acc);
+          }
+        }
+        tc_fence_before();
+      } else {
+        float ks_next = load_ks(0);  // E4M3: one tile ahead of its use
+        for (int n = 0; n < n2; ++n) {
+          const int bb = n & 1;
+          float sl = p.scale_log2;
+          if (FP8) {
+            sl *= ks_next;
+            ks_next = load_ks(n + 1);
+          }
+          if (!mbar_wait(&s2_full[bb], (n >> 1) & 1)) break;
+          tc_fence_after();
+          float acc[G];
+#pragma unroll
+          for (int q = 0; q < G; ++q) acc[q] = 0.f;
+#pragma unroll
+          for (int c = 0; c < N / 32; ++c) {
+            float x[32];
+            tmem_ld32(tmem + lane_base + bb * N + 32 * c, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              acc[(32 * c + i) / kH] += fast_exp2(x[i] * sl - lse2_s[32 * c + i]);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s2_empty[bb]);
+          emit(n, acc);
         }
       }
       asm volatile("bar.sync 2, 128;" ::: "memory");
@@ -977,8 +1069,19 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         }
         const float* po = p.part_o + ((long long)grp * ns * N + r) * 128 + d;
         float acc = 0.f;
-        constexpr int kLoadBatch = 16;   // the splits' values of element d, loaded together
-        for (int sp0 = 0; sp0 < ns; sp0 += kLoadBatch) {
+        int sp_first = 0;
+        if (r == split) {  // the prefetched splits
+#pragma unroll
+          for (int k = 0; k < kPre; ++k) {
+            if (k >= ns) break;
+            const float2 v = ml_s[r * ns + k];
+            const float f = (v.x == kNegInf) ? 0.f : fast_exp2(v.x - l2);
+            acc += f * pre[k];
+          }
+          sp_first = kPre;
+        }
+        constexpr int kLoadBatch = 24;   // the splits' values of element d, loaded together
+        for (int sp0 = sp_first; sp0 < ns; sp0 += kLoadBatch) {
           float x[kLoadBatch];
 #pragma unroll
           for (int k = 0; k < kLoadBatch; ++k)
@@ -999,20 +1102,26 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   __syncthreads();
 
   // ------------------------------------------ selection (whole group)
-  // The k-th largest score pattern tau, as in select_topk_kernel, in two group
-  // barriers.  (1) Once the level-1 histogram (bits [30:20], built by the
-  // score pass) is complete, every CTA finds the bin b1 holding the k-th
-  // candidate, counts its split's candidates above b1 and writes the ones in
-  // b1 to its slice of the row's list.  (2) Once every split has done so, every
-  // CTA loads the row's whole b1 list (split order) and finds tau and the
-  // number of ties to keep from two more digit levels (bits [19:9], [8:0]) in
-  // shared memory; the list prefix before its own slice gives the survivors of
-  // the lower splits, and it writes its own survivors in position order.
+  // The k-th largest score pattern tau, as in select_topk_kernel.  Once the
+  // level-1 histogram (bits [30:20], built by the score pass) is complete,
+  // every CTA finds the bin b1 holding the k-th candidate; then it needs the
+  // row's candidates in b1 to find tau and the number of ties to keep from two
+  // more digit levels (bits [19:9], [8:0]) in shared memory.
+  //   sel_rowscan: every split's score pass also wrote its scores into the
+  //     row's global copy, so each CTA bulk-copies the whole row into shared
+  //     memory (during the bin search) and picks out the b1 candidates itself
+  //     -- no third barrier.
+  //   otherwise: each CTA counts its split's candidates above b1, writes the
+  //     ones in b1 to its slice of a row list, and after a third group barrier
+  //     loads the row's whole list (split order).
+  // Either way the survivors of the lower splits follow, and each CTA writes
+  // its own split's survivors in position order.
   if (p.fuse_select) {
     const unsigned* segu = reinterpret_cast<const unsigned*>(seg);
-    unsigned* list_s = reinterpret_cast<unsigned*>(smem);                 // the row's b1 list
+    unsigned* list_s = reinterpret_cast<unsigned*>(smem);  // the row's b1 list, or the row
     unsigned* h = reinterpret_cast<unsigned*>(smem + SM::kSelWorkOff);    // 2048 counters
     int* off_s = reinterpret_cast<int*>(smem + SM::kSelWorkOff + 8192);   // [ns + 1] list offsets
+    uint64_t* row_bar = kv2_full + 2 * S2 + 8;
     auto row_of = [&](int q) { return (long long)b * p.T + t0 + q; };
     auto nc_of = [&](int q) { return p.qpos0 + t0 + q - p.window + 1; };
     auto active = [&](int q) { return t0 + q < p.T && nc_of(q) > p.topk && p.topk > 0; };
@@ -1026,135 +1135,217 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       give_up();
       return;
     }
+    if (!p.sel_rowscan) {
 #pragma unroll 1
-    for (int q = 0; q < G; ++q)
-      if (active(q)) {
-        sel_find_bin_global<kThreads, 2048>(p.hist + row_of(q) * kHistBins, p.topk, s_res, s_tmp);
-        const unsigned b1 = (unsigned)s_res[0];
-        if (threadIdx.x == 0) {
-          s_prefix[q] = s_res[0];
-          s_need[q] = s_res[1];
-        }
-        // this split's candidates above b1 and in b1, per warp-contiguous part
-        const int n = nseg_of(q);
-        const int wseg = (n + W - 1) / W;
-        const int w0 = min(n, warp * wseg), w1 = min(n, w0 + wseg);
-        int n_gt = 0, n_in = 0;
-        for (int base = w0; base < w1; base += 32) {
-          const int u = base + lane;
-          const unsigned d = u < w1 ? (segu[q * p.split_keys + u] >> 20) : 0u;
-          n_gt += __popc(__ballot_sync(0xffffffffu, u < w1 && d > b1));
-          n_in += __popc(__ballot_sync(0xffffffffu, u < w1 && d == b1));
-        }
-        if (lane == 0) {
-          s_wg[q][warp] = n_gt;
-          s_we[q][warp] = n_in;
-        }
-        __syncthreads();
-        int in_before = 0, gt_tot = 0, in_tot = 0;
-        for (int w = 0; w < W; ++w) {
-          if (w < warp) in_before += s_we[q][w];
-          gt_tot += s_wg[q][w];
-          in_tot += s_we[q][w];
-        }
-        if (threadIdx.x == 0) p.sel_cnt[row_of(q) * ns + split] = make_int2(gt_tot, in_tot);
-        unsigned* lg = list_g(q, split);
-        for (int base = w0; base < w1; base += 32) {
-          const int u = base + lane;
-          const unsigned v = u < w1 ? segu[q * p.split_keys + u] : 0u;
-          const bool in = u < w1 && (v >> 20) == b1;
-          const unsigned m = __ballot_sync(0xffffffffu, in);
-          if (in) lg[in_before + __popc(m & ((1u << lane) - 1u))] = v;
-          in_before += __popc(m);
-        }
-        __syncthreads();  // s_res / s_w* are reused by the next row
-      }
-    // every split's counts and b1 slice are out
-    if (!group_arrive_wait(gsync + 2, target, p.wait_limit_ns)) {
-      give_up();
-      return;
-    }
-#pragma unroll 1
-    for (int q = 0; q < G; ++q)
-      if (active(q)) {
-        // list offsets of the splits, and this split's survivors-above-b1 base
-        int2 c = make_int2(0, 0);
-        if (threadIdx.x < ns) c = __ldcg(p.sel_cnt + row_of(q) * ns + threadIdx.x);
-        int in_ex, gt_ex;
-        const int m = sel_block_scan<kThreads>(c.y, in_ex, s_tmp);
-        sel_block_scan<kThreads>(c.x, gt_ex, s_tmp);
-        if (threadIdx.x < ns) off_s[threadIdx.x] = in_ex;
-        if (threadIdx.x == ns) off_s[ns] = m;
-        if (threadIdx.x == split) {
-          s_base[0] = gt_ex;  // candidates above b1 in the lower splits
-          s_base[1] = in_ex;  // list index of this split's slice
-        }
-        for (int e = threadIdx.x; e < 2048; e += kThreads) h[e] = 0u;
-        __syncthreads();
-        // element e of the row's list: slice sp with off_s[sp] <= e < off_s[sp + 1]
-        const bool in_smem = m <= SM::kSelCap;
-        auto list_at = [&](int e) {
-          int lo = 0, hi = ns - 1;
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (off_s[mid] <= e) lo = mid;
-            else hi = mid - 1;
+      for (int q = 0; q < G; ++q)
+        if (active(q)) {
+          sel_find_bin_global<kThreads, 2048>(p.hist + row_of(q) * kHistBins, p.topk, s_res, s_tmp);
+          const unsigned b1 = (unsigned)s_res[0];
+          if (threadIdx.x == 0) {
+            s_prefix[q] = s_res[0];
+            s_need[q] = s_res[1];
           }
-          return __ldcg(list_g(q, lo) + (e - off_s[lo]));
-        };
-        if (in_smem) {
-          // kLoadBatch independent L2 loads in flight per thread (the list can
-          // hold thousands of entries: one round trip per entry would dominate)
-          constexpr int kLoadBatch = 8;
-          for (int e0 = threadIdx.x; e0 < m; e0 += kLoadBatch * kThreads) {
-            unsigned v[kLoadBatch];
-#pragma unroll
-            for (int u = 0; u < kLoadBatch; ++u) {
-              const int e = e0 + u * kThreads;
-              v[u] = e < m ? list_at(e) : 0u;
-            }
-#pragma unroll
-            for (int u = 0; u < kLoadBatch; ++u) {
-              const int e = e0 + u * kThreads;
-              if (e < m) list_s[e] = v[u];
-            }
+          // this split's candidates above b1 and in b1, per warp-contiguous part
+          const int n = nseg_of(q);
+          const int wseg = (n + W - 1) / W;
+          const int w0 = min(n, warp * wseg), w1 = min(n, w0 + wseg);
+          int n_gt = 0, n_in = 0;
+          for (int base = w0; base < w1; base += 32) {
+            const int u = base + lane;
+            const unsigned d = u < w1 ? (segu[q * p.split_keys + u] >> 20) : 0u;
+            n_gt += __popc(__ballot_sync(0xffffffffu, u < w1 && d > b1));
+            n_in += __popc(__ballot_sync(0xffffffffu, u < w1 && d == b1));
           }
-        }
-        __syncthreads();
-        auto val = [&](int e) { return in_smem ? list_s[e] : list_at(e); };
-        // levels 2 and 3 -- bits [19:9], then [8:0], of the list's elements that
-        // share the digits found so far -- as one loop over the same code (it
-        // runs once per launch, so every distinct instruction is fetched cold)
-        unsigned tau = (unsigned)s_prefix[q];
-        int need_tau = s_need[q];
-#pragma unroll 1
-        for (int lvl = 0; lvl < 2; ++lvl) {
-          const int shift = lvl == 0 ? 9 : 0, nbins = lvl == 0 ? 2048 : 512;
-          const int kept = lvl == 0 ? 20 : 9;   // bits above the digit: those found so far
-          if (lvl == 1) {
-            for (int e = threadIdx.x; e < 512; e += kThreads) h[e] = 0u;
-            __syncthreads();
-          }
-          for (int e = threadIdx.x; e < m; e += kThreads) {
-            const unsigned v = val(e);
-            hist_inc(h, (v >> shift) & (unsigned)(nbins - 1), (v >> kept) == tau);
+          if (lane == 0) {
+            s_wg[q][warp] = n_gt;
+            s_we[q][warp] = n_in;
           }
           __syncthreads();
-          sel_find_bin<kThreads>(h, nbins, need_tau, s_res, s_tmp);
-          tau = (tau << (lvl == 0 ? 11 : 9)) | (unsigned)s_res[0];
+          int in_before = 0, gt_tot = 0, in_tot = 0;
+          for (int w = 0; w < W; ++w) {
+            if (w < warp) in_before += s_we[q][w];
+            gt_tot += s_wg[q][w];
+            in_tot += s_we[q][w];
+          }
+          if (threadIdx.x == 0) p.sel_cnt[row_of(q) * ns + split] = make_int2(gt_tot, in_tot);
+          unsigned* lg = list_g(q, split);
+          for (int base = w0; base < w1; base += 32) {
+            const int u = base + lane;
+            const unsigned v = u < w1 ? segu[q * p.split_keys + u] : 0u;
+            const bool in = u < w1 && (v >> 20) == b1;
+            const unsigned m = __ballot_sync(0xffffffffu, in);
+            if (in) lg[in_before + __popc(m & ((1u << lane) - 1u))] = v;
+            in_before += __popc(m);
+          }
+          __syncthreads();  // s_res / s_w* are reused by the next row
+        }
+      // every split's counts and b1 slice are out
+      if (!group_arrive_wait(gsync + 2, target, p.wait_limit_ns)) {
+        give_up();
+        return;
+      }
+    }
+    uint32_t row_phase = 0;
+#pragma unroll 1
+    for (int q = 0; q < G; ++q)
+      if (active(q)) {
+        // tau (the k-th largest score pattern), need_tau (how many of the
+        // candidates equal to it are kept), and the lower splits' survivors:
+        // a_tot above tau (plus s_base[0]) and tie_tot equal to it
+        unsigned tau = 0u;
+        int need_tau = 0, a_tot = 0, tie_tot = 0;
+        if (p.sel_rowscan) {
+          // the row copy in shared memory (every candidate at its position):
+          // two passes over it, each building the next digit's histogram
+          const int n = (int)nc_of(q);
+          const int n4 = (n + 3) >> 2;
+          if (threadIdx.x == 0) {
+            fence_proxy_async_global();  // the other splits' scores, acquired at the barrier
+            fence_proxy_async_smem();    // earlier generic use of the destination
+            const uint32_t bytes = (uint32_t)n4 * 16u;
+            mbar_arrive_expect_tx(row_bar, bytes);
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(
+                p.sel_list + row_of(q) * (long long)ns * p.split_keys);
+            for (uint32_t o = 0; o < bytes; o += 32768u)
+              bulk_load_1d(smem + o, src + o, min(32768u, bytes - o), row_bar);
+          }
+          for (int e = threadIdx.x; e < 2048; e += kThreads) h[e] = 0u;
+          sel_find_bin_global<kThreads, 2048>(p.hist + row_of(q) * kHistBins, p.topk, s_res, s_tmp);
+          const unsigned b1 = (unsigned)s_res[0];
+          const int need1 = s_res[1];
+          const bool landed = mbar_wait(row_bar, row_phase & 1u);
+          ++row_phase;
+          if (!__syncthreads_and(landed)) {  // the copy is not in flight any more only if it landed
+            give_up();
+            return;
+          }
+          const uint4* row4 = reinterpret_cast<const uint4*>(list_s);
+          // pass 1: bits [19:9] of the b1 candidates; the candidates above b1 below this split
+          int gt1 = 0;
+          for (int e4 = threadIdx.x; e4 < n4; e4 += kThreads) {
+            const uint4 v4 = row4[e4];
+            const unsigned vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int e = 4 * e4 + k;
+              const unsigned d = vv[k] >> 20;
+              gt1 += (e < n && e < k_lo && d > b1) ? 1 : 0;
+              hist_inc(h, (vv[k] >> 9) & 2047u, e < n && d == b1);
+            }
+          }
+          int ex;
+          const int gt1_tot = sel_block_scan<kThreads>(gt1, ex, s_tmp);  // also completes h
+          sel_find_bin<kThreads>(h, 2048, need1, s_res, s_tmp);
+          const unsigned b2 = (b1 << 11) | (unsigned)s_res[0];
+          const int need2 = s_res[1];
+          // pass 2: bits [8:0] of the candidates in b2 (h[0, 512)) and of those
+          // below this split (h[512, 1024)); the b1 candidates above b2 below it
+          for (int e = threadIdx.x; e < 1024; e += kThreads) h[e] = 0u;
+          __syncthreads();
+          int gt2 = 0;
+          for (int e4 = threadIdx.x; e4 < n4; e4 += kThreads) {
+            const uint4 v4 = row4[e4];
+            const unsigned vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int e = 4 * e4 + k;
+              const unsigned d = vv[k] >> 9;
+              const bool low = e < n && e < k_lo;
+              gt2 += (low && (d >> 11) == b1 && d > b2) ? 1 : 0;
+              hist_inc(h, vv[k] & 511u, e < n && d == b2);
+              hist_inc(h + 512, vv[k] & 511u, low && d == b2);
+            }
+          }
+          const int gt2_tot = sel_block_scan<kThreads>(gt2, ex, s_tmp);  // also completes h
+          sel_find_bin<kThreads>(h, 512, need2, s_res, s_tmp);
+          const int b3 = s_res[0];
+          tau = (b2 << 9) | (unsigned)b3;
           need_tau = s_res[1];
+          int a3 = 0;
+          for (int u = threadIdx.x; u < 512; u += kThreads) a3 += u > b3 ? (int)h[512 + u] : 0;
+          a_tot = gt1_tot + gt2_tot + sel_block_scan<kThreads>(a3, ex, s_tmp);
+          tie_tot = (int)h[512 + b3];
+          if (threadIdx.x == 0) s_base[0] = 0;
+        } else {
+          // list offsets of the splits, and this split's survivors-above-b1 base
+          int2 c = make_int2(0, 0);
+          if (threadIdx.x < ns) c = __ldcg(p.sel_cnt + row_of(q) * ns + threadIdx.x);
+          int in_ex, gt_ex;
+          const int m = sel_block_scan<kThreads>(c.y, in_ex, s_tmp);
+          sel_block_scan<kThreads>(c.x, gt_ex, s_tmp);
+          if (threadIdx.x < ns) off_s[threadIdx.x] = in_ex;
+          if (threadIdx.x == ns) off_s[ns] = m;
+          if (threadIdx.x == split) {
+            s_base[0] = gt_ex;  // candidates above b1 in the lower splits
+            s_base[1] = in_ex;  // list index of this split's slice
+          }
+          for (int e = threadIdx.x; e < 2048; e += kThreads) h[e] = 0u;
+          __syncthreads();
+          const bool in_smem = m <= SM::kSelCap;
+          const int own = s_base[1];
+          tau = (unsigned)s_prefix[q];
+          need_tau = s_need[q];
+          // element e of the list: slice sp with off_s[sp] <= e < off_s[sp + 1]
+          auto list_at = [&](int e) {
+            int lo = 0, hi = ns - 1;
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if (off_s[mid] <= e) lo = mid;
+              else hi = mid - 1;
+            }
+            return __ldcg(list_g(q, lo) + (e - off_s[lo]));
+          };
+          if (in_smem) {
+            // kLoadBatch independent L2 loads in flight per thread (the list can
+            // hold thousands of entries: one round trip per entry would dominate)
+            constexpr int kLoadBatch = 8;
+            for (int e0 = threadIdx.x; e0 < m; e0 += kLoadBatch * kThreads) {
+              unsigned v[kLoadBatch];
+#pragma unroll
+              for (int u = 0; u < kLoadBatch; ++u) {
+                const int e = e0 + u * kThreads;
+                v[u] = e < m ? list_at(e) : 0u;
+              }
+#pragma unroll
+              for (int u = 0; u < kLoadBatch; ++u) {
+                const int e = e0 + u * kThreads;
+                if (e < m) list_s[e] = v[u];
+              }
+            }
+            __syncthreads();
+          }
+          auto val = [&](int e) { return in_smem ? list_s[e] : list_at(e); };
+          // levels 2 and 3 -- bits [19:9], then [8:0], of the list's elements that
+          // share the digits found so far -- as one loop over the same code (it
+          // runs once per launch, so every distinct instruction is fetched cold)
+#pragma unroll 1
+          for (int lvl = 0; lvl < 2; ++lvl) {
+            const int shift = lvl == 0 ? 9 : 0, nbins = lvl == 0 ? 2048 : 512;
+            const int kept = lvl == 0 ? 20 : 9;   // bits above the digit: those found so far
+            if (lvl == 1) {
+              for (int e = threadIdx.x; e < 512; e += kThreads) h[e] = 0u;
+              __syncthreads();
+            }
+            for (int e = threadIdx.x; e < m; e += kThreads) {
+              const unsigned v = val(e);
+              hist_inc(h, (v >> shift) & (unsigned)(nbins - 1), (v >> kept) == tau);
+            }
+            __syncthreads();
+            sel_find_bin<kThreads>(h, nbins, need_tau, s_res, s_tmp);
+            tau = (tau << (lvl == 0 ? 11 : 9)) | (unsigned)s_res[0];
+            need_tau = s_res[1];
+          }
+          // survivors of the lower splits' b1 slices: above tau, and ties
+          int a = 0, tie = 0;
+          for (int e = threadIdx.x; e < own; e += kThreads) {
+            const unsigned v = val(e);
+            a += v > tau;
+            tie += v == tau;
+          }
+          int a_ex, tie_ex;
+          a_tot = sel_block_scan<kThreads>(a, a_ex, s_tmp);
+          tie_tot = sel_block_scan<kThreads>(tie, tie_ex, s_tmp);
         }
-        // survivors of the lower splits' b1 slices: above tau, and ties
-        const int own = s_base[1];
-        int a = 0, tie = 0;
-        for (int e = threadIdx.x; e < own; e += kThreads) {
-          const unsigned v = val(e);
-          a += v > tau;
-          tie += v == tau;
-        }
-        int a_ex, tie_ex;
-        const int a_tot = sel_block_scan<kThreads>(a, a_ex, s_tmp);
-        const int tie_tot = sel_block_scan<kThreads>(tie, tie_ex, s_tmp);
         // this split's survivors, per warp-contiguous part: v > tau, v == tau
         const int n = nseg_of(q);
         const int wseg = (n + W - 1) / W;

@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     bridge_gemm_kernel(const __grid_constant__ CUtensorMap xmap,
                        const __grid_constant__ CUtensorMap wmap, const BridgeParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBrBarOff);
   uint64_t* empty = full + kBrStages;
   uint64_t* acc_full = empty + kBrStages;   // [2]

@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   static_assert(SM::kBytes <= 232448, "shared memory per CTA");
   constexpr int kTokPerOwner = SM::kTokPerOwner;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
   uint64_t* empty = full + kBsStages;
   uint64_t* done = empty + kBsStages;

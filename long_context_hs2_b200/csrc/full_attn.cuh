@@ -44,11 +44,16 @@ struct FullAttnParams {
   // fused tcgen05 pass only: per-group arrival counters (zeroed before the
   // launch), and the selection outputs when the selection is fused too
   unsigned* grp_sync;            // [groups][8]
-  unsigned* sel_list;            // [B*T][splits][split_keys] candidate scores in the level-1 bin
+  // [B*T][splits * split_keys]: with sel_rowscan, the row's candidate scores at
+  // their positions; else split sp's slice holds its candidates in the level-1 bin
+  unsigned* sel_list;
   int2* sel_cnt;                 // [B*T][splits] candidates above / in the level-1 bin per split
   int32_t* idx;                  // [B*T][slots]
   int32_t* n_sel;                // [B*T]
   int topk, slots, fuse_select;
+  // fused selection with every CTA holding its rows' whole score rows in shared
+  // memory (two group barriers), instead of exchanging level-1 bin lists (three)
+  int sel_rowscan;
   // the group barriers' wait limit, and arrivals they wait for beyond the
   // group's CTA count (non-zero only under fault injection)
   unsigned long long wait_limit_ns;
@@ -88,10 +93,6 @@ struct FullAttnSmem {
   static constexpr int kScoreBarOff = kScoreLseOff + kRows * 4;
   static constexpr int kScoreBytes = kScoreBarOff + 2 * kScoreStages * 8 + 1024;
 };
-
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
-}
 
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
