@@ -76,7 +76,7 @@ struct TcSmem {
   static constexpr int kNumBars = 3 * kStages + 13 + 2 * kNP;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBar2Off = kSlotOff + 16;         // fused kernel: score-pass barriers
-  static constexpr int kNumBars2 = 17;  // + the row copy of the fused selection
+  static constexpr int kNumBars2 = 16;
   // retained tiles' references (16-byte aligned: read as float4)
   static constexpr int kMhistOff = (kBar2Off + kNumBars2 * 8 + 15) / 16 * 16;
   static constexpr int kMhistBytes = N == 32 ? 15 * N * 4 : 0;
@@ -799,7 +799,6 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       mbar_init(&k2_full[i], 4);
       mbar_init(&k2_free[i], 1);
     }
-    mbar_init(k2_free + 2, 1);  // the fused selection's row copy
     fence_mbar_init();
   }
   if (threadIdx.x / 32 == 1) {
@@ -972,15 +971,9 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         for (int q = 0; q < G; ++q) {
           const int t = t0 + q;
           const bool cand = t < p.T && j <= p.qpos0 + t - p.window;
-          if (cand) {  // the fused selection reads the shared-memory copy (and the row copy)
-            if (p.fuse_select) {
-              seg[q * p.split_keys + (int)(j - k_lo)] = acc[q];
-              if (p.sel_rowscan)
-                p.sel_list[((long long)b * p.T + t) * ns * p.split_keys + j] =
-                    __float_as_uint(acc[q]);
-            } else {
-              p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
-            }
+          if (cand) {  // the fused selection reads the shared-memory copy only
+            if (p.fuse_select) seg[q * p.split_keys + (int)(j - k_lo)] = acc[q];
+            else p.score[((long long)b * p.T + t) * p.L + j] = acc[q];
           }
           hist_inc(hist_s + q * kHistBins, __float_as_uint(acc[q]) >> kHistShift, cand);
         }
@@ -1102,26 +1095,23 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   __syncthreads();
 
   // ------------------------------------------ selection (whole group)
-  // The k-th largest score pattern tau, as in select_topk_kernel.  Once the
-  // level-1 histogram (bits [30:20], built by the score pass) is complete,
-  // every CTA finds the bin b1 holding the k-th candidate; then it needs the
-  // row's candidates in b1 to find tau and the number of ties to keep from two
-  // more digit levels (bits [19:9], [8:0]) in shared memory.
-  //   sel_rowscan: every split's score pass also wrote its scores into the
-  //     row's global copy, so each CTA bulk-copies the whole row into shared
-  //     memory (during the bin search) and picks out the b1 candidates itself
-  //     -- no third barrier.
-  //   otherwise: each CTA counts its split's candidates above b1, writes the
-  //     ones in b1 to its slice of a row list, and after a third group barrier
-  //     loads the row's whole list (split order).
-  // Either way the survivors of the lower splits follow, and each CTA writes
-  // its own split's survivors in position order.
+  // The k-th largest score pattern tau, as in select_topk_kernel, in two group
+  // barriers.  (1) Once the level-1 histogram (bits [30:20], built by the
+  // score pass) is complete, every CTA finds the bin b1 holding the k-th
+  // candidate, counts its split's candidates above b1 and writes the ones in
+  // b1 to its slice of the row's list.  (2) Once every split has done so, every
+  // CTA loads the row's whole b1 list (split order) and finds tau and the
+  // number of ties to keep from two more digit levels (bits [19:9], [8:0]) in
+  // shared memory; the list prefix before its own slice gives the survivors of
+  // the lower splits, and it writes its own survivors in position order.  The
+  // chain runs once per launch, after the streaming: the in-list digit searches
+  // are one warp's (no block-wide scans), and every reduction one block barrier.
   if (p.fuse_select) {
     const unsigned* segu = reinterpret_cast<const unsigned*>(seg);
-    unsigned* list_s = reinterpret_cast<unsigned*>(smem);  // the row's b1 list, or the row
+    unsigned* list_s = reinterpret_cast<unsigned*>(smem);                 // the row's b1 list
     unsigned* h = reinterpret_cast<unsigned*>(smem + SM::kSelWorkOff);    // 2048 counters
     int* off_s = reinterpret_cast<int*>(smem + SM::kSelWorkOff + 8192);   // [ns + 1] list offsets
-    uint64_t* row_bar = kv2_full + 2 * S2 + 8;
+    __shared__ int s_red[2][16];
     auto row_of = [&](int q) { return (long long)b * p.T + t0 + q; };
     auto nc_of = [&](int q) { return p.qpos0 + t0 + q - p.window + 1; };
     auto active = [&](int q) { return t0 + q < p.T && nc_of(q) > p.topk && p.topk > 0; };
@@ -1131,221 +1121,177 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     auto list_g = [&](int q, int sp) {
       return p.sel_list + (row_of(q) * ns + sp) * (long long)p.split_keys;
     };
+    // block totals of two counts (one block barrier; s_red is free again after
+    // the caller's next barrier)
+    auto block_sum2 = [&](int x, int y, int& xt, int& yt) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        x += __shfl_xor_sync(0xffffffffu, x, o);
+        y += __shfl_xor_sync(0xffffffffu, y, o);
+      }
+      if (lane == 0) {
+        s_red[0][warp] = x;
+        s_red[1][warp] = y;
+      }
+      __syncthreads();
+      xt = 0;
+      yt = 0;
+      for (int w = 0; w < W; ++w) {
+        xt += s_red[0][w];
+        yt += s_red[1][w];
+      }
+    };
     if (!group_arrive_wait(gsync + 1, target, p.wait_limit_ns)) {  // level-1 counts complete
       give_up();
       return;
     }
-    if (!p.sel_rowscan) {
-#pragma unroll 1
-      for (int q = 0; q < G; ++q)
-        if (active(q)) {
-          sel_find_bin_global<kThreads, 2048>(p.hist + row_of(q) * kHistBins, p.topk, s_res, s_tmp);
-          const unsigned b1 = (unsigned)s_res[0];
-          if (threadIdx.x == 0) {
-            s_prefix[q] = s_res[0];
-            s_need[q] = s_res[1];
-          }
-          // this split's candidates above b1 and in b1, per warp-contiguous part
-          const int n = nseg_of(q);
-          const int wseg = (n + W - 1) / W;
-          const int w0 = min(n, warp * wseg), w1 = min(n, w0 + wseg);
-          int n_gt = 0, n_in = 0;
-          for (int base = w0; base < w1; base += 32) {
-            const int u = base + lane;
-            const unsigned d = u < w1 ? (segu[q * p.split_keys + u] >> 20) : 0u;
-            n_gt += __popc(__ballot_sync(0xffffffffu, u < w1 && d > b1));
-            n_in += __popc(__ballot_sync(0xffffffffu, u < w1 && d == b1));
-          }
-          if (lane == 0) {
-            s_wg[q][warp] = n_gt;
-            s_we[q][warp] = n_in;
-          }
-          __syncthreads();
-          int in_before = 0, gt_tot = 0, in_tot = 0;
-          for (int w = 0; w < W; ++w) {
-            if (w < warp) in_before += s_we[q][w];
-            gt_tot += s_wg[q][w];
-            in_tot += s_we[q][w];
-          }
-          if (threadIdx.x == 0) p.sel_cnt[row_of(q) * ns + split] = make_int2(gt_tot, in_tot);
-          unsigned* lg = list_g(q, split);
-          for (int base = w0; base < w1; base += 32) {
-            const int u = base + lane;
-            const unsigned v = u < w1 ? segu[q * p.split_keys + u] : 0u;
-            const bool in = u < w1 && (v >> 20) == b1;
-            const unsigned m = __ballot_sync(0xffffffffu, in);
-            if (in) lg[in_before + __popc(m & ((1u << lane) - 1u))] = v;
-            in_before += __popc(m);
-          }
-          __syncthreads();  // s_res / s_w* are reused by the next row
-        }
-      // every split's counts and b1 slice are out
-      if (!group_arrive_wait(gsync + 2, target, p.wait_limit_ns)) {
-        give_up();
-        return;
-      }
-    }
-    uint32_t row_phase = 0;
 #pragma unroll 1
     for (int q = 0; q < G; ++q)
       if (active(q)) {
-        // tau (the k-th largest score pattern), need_tau (how many of the
-        // candidates equal to it are kept), and the lower splits' survivors:
-        // a_tot above tau (plus s_base[0]) and tie_tot equal to it
-        unsigned tau = 0u;
-        int need_tau = 0, a_tot = 0, tie_tot = 0;
-        if (p.sel_rowscan) {
-          // the row copy in shared memory (every candidate at its position):
-          // two passes over it, each building the next digit's histogram
-          const int n = (int)nc_of(q);
-          const int n4 = (n + 3) >> 2;
-          if (threadIdx.x == 0) {
-            fence_proxy_async_global();  // the other splits' scores, acquired at the barrier
-            fence_proxy_async_smem();    // earlier generic use of the destination
-            const uint32_t bytes = (uint32_t)n4 * 16u;
-            mbar_arrive_expect_tx(row_bar, bytes);
-            const uint8_t* src = reinterpret_cast<const uint8_t*>(
-                p.sel_list + row_of(q) * (long long)ns * p.split_keys);
-            for (uint32_t o = 0; o < bytes; o += 32768u)
-              bulk_load_1d(smem + o, src + o, min(32768u, bytes - o), row_bar);
-          }
-          for (int e = threadIdx.x; e < 2048; e += kThreads) h[e] = 0u;
-          sel_find_bin_global<kThreads, 2048>(p.hist + row_of(q) * kHistBins, p.topk, s_res, s_tmp);
-          const unsigned b1 = (unsigned)s_res[0];
-          const int need1 = s_res[1];
-          const bool landed = mbar_wait(row_bar, row_phase & 1u);
-          ++row_phase;
-          if (!__syncthreads_and(landed)) {  // the copy is not in flight any more only if it landed
-            give_up();
-            return;
-          }
-          const uint4* row4 = reinterpret_cast<const uint4*>(list_s);
-          // pass 1: bits [19:9] of the b1 candidates; the candidates above b1 below this split
-          int gt1 = 0;
-          for (int e4 = threadIdx.x; e4 < n4; e4 += kThreads) {
-            const uint4 v4 = row4[e4];
-            const unsigned vv[4] = {v4.x, v4.y, v4.z, v4.w};
+        sel_find_bin_global<kThreads, 2048>(p.hist + row_of(q) * kHistBins, p.topk, s_res, s_tmp);
+        const unsigned b1 = (unsigned)s_res[0];
+        if (threadIdx.x == 0) {
+          s_prefix[q] = s_res[0];
+          s_need[q] = s_res[1];
+        }
+        // this split's candidates above b1 and in b1, per warp-contiguous part
+        const int n = nseg_of(q);
+        const int wseg = (n + W - 1) / W;
+        const int w0 = min(n, warp * wseg), w1 = min(n, w0 + wseg);
+        int n_gt = 0, n_in = 0;
+        for (int base = w0; base < w1; base += 32) {
+          const int u = base + lane;
+          const unsigned d = u < w1 ? (segu[q * p.split_keys + u] >> 20) : 0u;
+          n_gt += __popc(__ballot_sync(0xffffffffu, u < w1 && d > b1));
+          n_in += __popc(__ballot_sync(0xffffffffu, u < w1 && d == b1));
+        }
+        if (lane == 0) {
+          s_wg[q][warp] = n_gt;
+          s_we[q][warp] = n_in;
+        }
+        __syncthreads();
+        int in_before = 0, gt_tot = 0, in_tot = 0;
+        for (int w = 0; w < W; ++w) {
+          if (w < warp) in_before += s_we[q][w];
+          gt_tot += s_wg[q][w];
+          in_tot += s_we[q][w];
+        }
+        if (threadIdx.x == 0) p.sel_cnt[row_of(q) * ns + split] = make_int2(gt_tot, in_tot);
+        unsigned* lg = list_g(q, split);
+        for (int base = w0; base < w1; base += 32) {
+          const int u = base + lane;
+          const unsigned v = u < w1 ? segu[q * p.split_keys + u] : 0u;
+          const bool in = u < w1 && (v >> 20) == b1;
+          const unsigned m = __ballot_sync(0xffffffffu, in);
+          if (in) lg[in_before + __popc(m & ((1u << lane) - 1u))] = v;
+          in_before += __popc(m);
+        }
+        __syncthreads();  // s_res / s_w* are reused by the next row
+      }
+    // every split's counts and b1 slice are out
+    if (!group_arrive_wait(gsync + 2, target, p.wait_limit_ns)) {
+      give_up();
+      return;
+    }
+#pragma unroll 1
+    for (int q = 0; q < G; ++q)
+      if (active(q)) {
+        // list offsets of the splits, and this split's survivors-above-b1 base
+        if (ns <= 32) {  // one warp scans the splits' counts
+          if (warp == 0) {
+            int2 c = make_int2(0, 0);
+            if (lane < ns) c = __ldcg(p.sel_cnt + row_of(q) * ns + lane);
+            int ix = c.y, gx = c.x;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int e = 4 * e4 + k;
-              const unsigned d = vv[k] >> 20;
-              gt1 += (e < n && e < k_lo && d > b1) ? 1 : 0;
-              hist_inc(h, (vv[k] >> 9) & 2047u, e < n && d == b1);
+            for (int o = 1; o < 32; o <<= 1) {
+              const int yi = __shfl_up_sync(0xffffffffu, ix, o);
+              const int yg = __shfl_up_sync(0xffffffffu, gx, o);
+              if (lane >= o) {
+                ix += yi;
+                gx += yg;
+              }
+            }
+            if (lane < ns) off_s[lane] = ix - c.y;
+            if (lane == ns - 1) off_s[ns] = ix;
+            if (lane == split) {
+              s_base[0] = gx - c.x;  // candidates above b1 in the lower splits
+              s_base[1] = ix - c.y;  // list index of this split's slice
             }
           }
-          int ex;
-          const int gt1_tot = sel_block_scan<kThreads>(gt1, ex, s_tmp);  // also completes h
-          sel_find_bin<kThreads>(h, 2048, need1, s_res, s_tmp);
-          const unsigned b2 = (b1 << 11) | (unsigned)s_res[0];
-          const int need2 = s_res[1];
-          // pass 2: bits [8:0] of the candidates in b2 (h[0, 512)) and of those
-          // below this split (h[512, 1024)); the b1 candidates above b2 below it
-          for (int e = threadIdx.x; e < 1024; e += kThreads) h[e] = 0u;
-          __syncthreads();
-          int gt2 = 0;
-          for (int e4 = threadIdx.x; e4 < n4; e4 += kThreads) {
-            const uint4 v4 = row4[e4];
-            const unsigned vv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int e = 4 * e4 + k;
-              const unsigned d = vv[k] >> 9;
-              const bool low = e < n && e < k_lo;
-              gt2 += (low && (d >> 11) == b1 && d > b2) ? 1 : 0;
-              hist_inc(h, vv[k] & 511u, e < n && d == b2);
-              hist_inc(h + 512, vv[k] & 511u, low && d == b2);
-            }
-          }
-          const int gt2_tot = sel_block_scan<kThreads>(gt2, ex, s_tmp);  // also completes h
-          sel_find_bin<kThreads>(h, 512, need2, s_res, s_tmp);
-          const int b3 = s_res[0];
-          tau = (b2 << 9) | (unsigned)b3;
-          need_tau = s_res[1];
-          int a3 = 0;
-          for (int u = threadIdx.x; u < 512; u += kThreads) a3 += u > b3 ? (int)h[512 + u] : 0;
-          a_tot = gt1_tot + gt2_tot + sel_block_scan<kThreads>(a3, ex, s_tmp);
-          tie_tot = (int)h[512 + b3];
-          if (threadIdx.x == 0) s_base[0] = 0;
         } else {
-          // list offsets of the splits, and this split's survivors-above-b1 base
           int2 c = make_int2(0, 0);
           if (threadIdx.x < ns) c = __ldcg(p.sel_cnt + row_of(q) * ns + threadIdx.x);
           int in_ex, gt_ex;
-          const int m = sel_block_scan<kThreads>(c.y, in_ex, s_tmp);
+          const int m_all = sel_block_scan<kThreads>(c.y, in_ex, s_tmp);
           sel_block_scan<kThreads>(c.x, gt_ex, s_tmp);
           if (threadIdx.x < ns) off_s[threadIdx.x] = in_ex;
-          if (threadIdx.x == ns) off_s[ns] = m;
+          if (threadIdx.x == ns) off_s[ns] = m_all;
           if (threadIdx.x == split) {
-            s_base[0] = gt_ex;  // candidates above b1 in the lower splits
-            s_base[1] = in_ex;  // list index of this split's slice
+            s_base[0] = gt_ex;
+            s_base[1] = in_ex;
           }
-          for (int e = threadIdx.x; e < 2048; e += kThreads) h[e] = 0u;
-          __syncthreads();
-          const bool in_smem = m <= SM::kSelCap;
-          const int own = s_base[1];
-          tau = (unsigned)s_prefix[q];
-          need_tau = s_need[q];
-          // element e of the list: slice sp with off_s[sp] <= e < off_s[sp + 1]
-          auto list_at = [&](int e) {
-            int lo = 0, hi = ns - 1;
-            while (lo < hi) {
-              const int mid = (lo + hi + 1) >> 1;
-              if (off_s[mid] <= e) lo = mid;
-              else hi = mid - 1;
-            }
-            return __ldcg(list_g(q, lo) + (e - off_s[lo]));
-          };
-          if (in_smem) {
-            // kLoadBatch independent L2 loads in flight per thread (the list can
-            // hold thousands of entries: one round trip per entry would dominate)
-            constexpr int kLoadBatch = 8;
-            for (int e0 = threadIdx.x; e0 < m; e0 += kLoadBatch * kThreads) {
-              unsigned v[kLoadBatch];
-#pragma unroll
-              for (int u = 0; u < kLoadBatch; ++u) {
-                const int e = e0 + u * kThreads;
-                v[u] = e < m ? list_at(e) : 0u;
-              }
-#pragma unroll
-              for (int u = 0; u < kLoadBatch; ++u) {
-                const int e = e0 + u * kThreads;
-                if (e < m) list_s[e] = v[u];
-              }
-            }
-            __syncthreads();
-          }
-          auto val = [&](int e) { return in_smem ? list_s[e] : list_at(e); };
-          // levels 2 and 3 -- bits [19:9], then [8:0], of the list's elements that
-          // share the digits found so far -- as one loop over the same code (it
-          // runs once per launch, so every distinct instruction is fetched cold)
-#pragma unroll 1
-          for (int lvl = 0; lvl < 2; ++lvl) {
-            const int shift = lvl == 0 ? 9 : 0, nbins = lvl == 0 ? 2048 : 512;
-            const int kept = lvl == 0 ? 20 : 9;   // bits above the digit: those found so far
-            if (lvl == 1) {
-              for (int e = threadIdx.x; e < 512; e += kThreads) h[e] = 0u;
-              __syncthreads();
-            }
-            for (int e = threadIdx.x; e < m; e += kThreads) {
-              const unsigned v = val(e);
-              hist_inc(h, (v >> shift) & (unsigned)(nbins - 1), (v >> kept) == tau);
-            }
-            __syncthreads();
-            sel_find_bin<kThreads>(h, nbins, need_tau, s_res, s_tmp);
-            tau = (tau << (lvl == 0 ? 11 : 9)) | (unsigned)s_res[0];
-            need_tau = s_res[1];
-          }
-          // survivors of the lower splits' b1 slices: above tau, and ties
-          int a = 0, tie = 0;
-          for (int e = threadIdx.x; e < own; e += kThreads) {
-            const unsigned v = val(e);
-            a += v > tau;
-            tie += v == tau;
-          }
-          int a_ex, tie_ex;
-          a_tot = sel_block_scan<kThreads>(a, a_ex, s_tmp);
-          tie_tot = sel_block_scan<kThreads>(tie, tie_ex, s_tmp);
         }
+        for (int e = threadIdx.x; e < 2048; e += kThreads) h[e] = 0u;
+        __syncthreads();
+        const int m = off_s[ns];
+        const bool in_smem = m <= SM::kSelCap;
+        // element e of the row's list: slice sp with off_s[sp] <= e < off_s[sp + 1]
+        auto list_at = [&](int e) {
+          int lo = 0, hi = ns - 1;
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (off_s[mid] <= e) lo = mid;
+            else hi = mid - 1;
+          }
+          return __ldcg(list_g(q, lo) + (e - off_s[lo]));
+        };
+        if (in_smem) {
+          // the slices, one warp each at a time: all loads of a warp's slices
+          // are independent (a single L2 round trip for a decode row)
+          for (int sp = warp; sp < ns; sp += W) {
+            const int o = off_s[sp], cnt = off_s[sp + 1] - o;
+            const unsigned* src = list_g(q, sp);
+            for (int e = lane; e < cnt; e += 32) list_s[o + e] = __ldcg(src + e);
+          }
+          __syncthreads();
+        }
+        auto val = [&](int e) { return in_smem ? list_s[e] : list_at(e); };
+        // levels 2 and 3 -- bits [19:9], then [8:0], of the list's elements that
+        // share the digits found so far -- as one loop over the same code (it
+        // runs once per launch, so every distinct instruction is fetched cold)
+        unsigned tau = (unsigned)s_prefix[q];
+        int need_tau = s_need[q];
+#pragma unroll 1
+        for (int lvl = 0; lvl < 2; ++lvl) {
+          const int shift = lvl == 0 ? 9 : 0;
+          const int kept = lvl == 0 ? 20 : 9;   // bits above the digit: those found so far
+          if (lvl == 1) {
+            for (int e = threadIdx.x; e < 512; e += kThreads) h[e] = 0u;
+            __syncthreads();
+          }
+          for (int e = threadIdx.x; e < m; e += kThreads) {
+            const unsigned v = val(e);
+            hist_inc(h, (v >> shift) & (lvl == 0 ? 2047u : 511u), (v >> kept) == tau);
+          }
+          __syncthreads();
+          if (warp == 0) {
+            if (lvl == 0) sel_find_bin_warp<2048>(h, need_tau, s_res);
+            else sel_find_bin_warp<512>(h, need_tau, s_res);
+          }
+          __syncthreads();
+          tau = (tau << (lvl == 0 ? 11 : 9)) | (unsigned)s_res[0];
+          need_tau = s_res[1];
+        }
+        // survivors of the lower splits' b1 slices: above tau, and ties
+        const int own = s_base[1];
+        int a = 0, tie = 0;
+        for (int e = threadIdx.x; e < own; e += kThreads) {
+          const unsigned v = val(e);
+          a += v > tau;
+          tie += v == tau;
+        }
+        int a_tot, tie_tot;
+        block_sum2(a, tie, a_tot, tie_tot);
         // this split's survivors, per warp-contiguous part: v > tau, v == tau
         const int n = nseg_of(q);
         const int wseg = (n + W - 1) / W;

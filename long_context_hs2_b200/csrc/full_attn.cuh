@@ -44,16 +44,11 @@ struct FullAttnParams {
   // fused tcgen05 pass only: per-group arrival counters (zeroed before the
   // launch), and the selection outputs when the selection is fused too
   unsigned* grp_sync;            // [groups][8]
-  // [B*T][splits * split_keys]: with sel_rowscan, the row's candidate scores at
-  // their positions; else split sp's slice holds its candidates in the level-1 bin
-  unsigned* sel_list;
+  unsigned* sel_list;            // [B*T][splits][split_keys] candidate scores in the level-1 bin
   int2* sel_cnt;                 // [B*T][splits] candidates above / in the level-1 bin per split
   int32_t* idx;                  // [B*T][slots]
   int32_t* n_sel;                // [B*T]
   int topk, slots, fuse_select;
-  // fused selection with every CTA holding its rows' whole score rows in shared
-  // memory (two group barriers), instead of exchanging level-1 bin lists (three)
-  int sel_rowscan;
   // the group barriers' wait limit, and arrivals they wait for beyond the
   // group's CTA count (non-zero only under fault injection)
   unsigned long long wait_limit_ns;

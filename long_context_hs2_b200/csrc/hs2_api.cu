@@ -321,9 +321,6 @@ hs2_status run_fused_tc(const CUtensorMap& km, const CUtensorMap& vm, FullAttnPa
   // without token_select the caller runs another selection on the scores
   fp.fuse_select = token_select && (long long)fp.G * fp.split_keys * 4 <= SM::kNP * SM::kPBytes &&
                    pl.n_splits <= 256;
-  // every CTA then copies each of its rows' candidate scores whole into the
-  // tile ring when a row (16-byte rounded) leaves at least 4 KB of it free
-  fp.sel_rowscan = fp.fuse_select && (fp.L + 3) / 4 * 16 <= SM::kSelWorkOff - 4096;
   // the logits of every tile stay in TMEM for the score pass when a split has
   // at most kTcRetainTiles tiles
   const bool retain = (fp.split_keys + kTcKeys - 1) / kTcKeys <= kTcRetainTiles;
@@ -542,7 +539,6 @@ hs2_status setup_full(const void* Q, const hs2_kv_cache* kv, int B, int T, int64
   fp.topk = topk;
   fp.slots = topk + window;
   fp.fuse_select = 0;
-  fp.sel_rowscan = 0;
   fp.wait_limit_ns = t_wait_limit_ns;
   fp.barrier_extra = t_barrier_extra;
   fp.qpos0 = L - T;

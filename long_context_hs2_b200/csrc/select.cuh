@@ -167,6 +167,63 @@ __device__ __forceinline__ void sel_find_bin_global(const unsigned* hist, int k,
   __syncthreads();
 }
 
+// The same search over a shared-memory histogram by one warp (all 32 lanes;
+// a block barrier must follow before res is read), in short loops: the code
+// runs once per launch, when it is not in the instruction caches.  Lane l sums
+// the NB/32 bins below NB - l*NB/32 (16-byte loads), a warp scan from the top
+// finds the owner lane, and the whole warp then searches the owner's bins,
+// NB/1024 (at least one) per lane.
+template <int NB>
+__device__ __forceinline__ void sel_find_bin_warp(const unsigned* hist, int k, int* res) {
+  constexpr int PER = NB / 32;
+  constexpr int R = PER >= 32 ? PER / 32 : 1;
+  static_assert(PER % 4 == 0, "whole 16-byte groups per lane");
+  const int lane = threadIdx.x & 31;
+  const int lo = NB - (lane + 1) * PER;
+  int local = 0;
+#pragma unroll 1
+  for (int e = 0; e < PER; e += 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(hist + lo + e);
+    local += (int)(v.x + v.y + v.z + v.w);
+  }
+  int incl = local;  // lane 0 holds the highest bins
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned own = __ballot_sync(0xffffffffu, incl - local < k && k <= incl);
+  if (own == 0u) return;  // k above the histogram's total: res is left as it was
+  const int ol = __ffs((int)own) - 1;
+  const int above = __shfl_sync(0xffffffffu, incl - local, ol);
+  const int top = NB - 1 - ol * PER;  // the owner's highest bin
+  // lane j: the owner's bins top - j*R - r, r < R
+  int cnt = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    if (lane * R + r < PER) cnt += (int)hist[top - lane * R - r];
+  int inc2 = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc2, o);
+    if (lane >= o) inc2 += y;
+  }
+  if (above + inc2 - cnt < k && k <= above + inc2) {
+    int acc = above + inc2 - cnt;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int bin = top - lane * R - r;
+      const int c = (int)hist[bin];
+      if (acc + c >= k) {
+        res[0] = bin;
+        res[1] = k - acc;
+        break;
+      }
+      acc += c;
+    }
+  }
+}
+
 template <bool SMEM>
 __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectParams p) {
   __shared__ unsigned h2[2048];       // this CTA's level-2 histogram
