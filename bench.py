@@ -51,7 +51,90 @@ def parse():
     ap.add_argument("--only", choices=["append", "blocks", "configs", "decode_fp8_256k",
                                        "chunk_fp8_1m"], default=None,
                     help="run one section alone on one GPU and print its JSON (for profiling)")
+    ap.add_argument("--profile-case", choices=list(PROFILE_CASES), default=None,
+                    help="two untimed calls of one small case, for an ncu capture of its kernels")
     return ap.parse_args()
+
+
+# Small cases of the library's calls for ncu captures: inputs larger than L2
+# where DRAM figures matter, a few GB on the device at most.
+PROFILE_CASES = {
+    "decode_bf16": "hs2_full_attn_select on the 8 x 32K bf16 decode workload",
+    "decode_fp8": "hs2_full_attn_select on the 4 x 256K E4M3 decode workload",
+    "chunk_small": "hs2_full_attn_select on a 512-query chunk over 128K E4M3 tokens",
+    "sparse_chunk": "hs2_sparse_attn on a 1024-query chunk over 256K E4M3 tokens",
+    "bridge_append": "hs2_bridge_kv of 64 tokens into 6 layers' E4M3 caches",
+}
+
+
+def run_profile_case(name):
+    """Two calls of one PROFILE_CASES case, L2 flushed before each; exits non-zero
+    when the device status reports an error."""
+    import torch
+    import long_context_hs2_b200 as hs2
+    g = torch.Generator(device="cuda").manual_seed(1)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def l2_flush():
+        flush.zero_()
+        flush.view(torch.int64).amax()
+
+    def e4m3(n, D):
+        x = torch.randn(n, D, device="cuda", generator=g)
+        sc = x.abs().amax(1).clamp_min(1e-30) / 448.0 * (1 + torch.rand(n, device="cuda", generator=g) / 2)
+        return (x / sc[:, None]).to(torch.float8_e4m3fn).view(torch.uint8), sc.float()
+
+    def attn(wname, **kw):
+        wl = WORKLOADS[wname].resized(**kw) if kw else WORKLOADS[wname]
+        B, T, L, H, D = wl.B, wl.T, wl.L, wl.H, wl.D
+        q = torch.randn(B, T, H, D, device="cuda", generator=g).to(torch.bfloat16)
+        if wl.kv_dtype == "fp8":
+            k, ks = e4m3(B * L, D)
+            v, vs = e4m3(B * L, D)
+            kv, dt = hs2.kv_cache(k, v, ks, vs), hs2.HS2_KV_FP8_E4M3
+        else:
+            k = torch.randn(B * L, D, device="cuda", generator=g).to(torch.bfloat16)
+            v = torch.randn(B * L, D, device="cuda", generator=g).to(torch.bfloat16)
+            kv, dt = hs2.kv_cache(k, v), hs2.HS2_KV_BF16
+        slots = wl.topk + wl.window
+        nb = hs2.hs2_full_attn_select_workspace(B, T, L, H, D, wl.topk, wl.window, dt)
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        O = torch.empty(B, T, H, D, device="cuda")
+        idx = torch.empty(B, T, slots, dtype=torch.int32, device="cuda")
+        ns = torch.empty(B, T, dtype=torch.int32, device="cuda")
+        full = lambda: hs2.hs2_full_attn_select(q, kv, B, T, L, H, D, wl.scale, wl.topk,
+                                                wl.window, dt, O, None, idx, ns, ws, nb)
+        sparse = lambda: hs2.hs2_sparse_attn(q, kv, B, T, L, H, D, wl.scale, idx, ns, slots, dt, O)
+        return full, sparse
+
+    if name == "decode_bf16":
+        calls = [attn("decode_bf16_32k")[0]] * 2
+    elif name == "decode_fp8":
+        calls = [attn("decode_fp8_256k")[0]] * 2
+    elif name == "chunk_small":
+        calls = [attn("chunk_fp8_1m", T=512, L=131072)[0]] * 2
+    elif name == "sparse_chunk":
+        full, sparse = attn("chunk_fp8_1m", T=1024, L=262144)
+        calls = [full, sparse, sparse]
+    else:  # bridge_append
+        T, hidden, nl, D, rows = 64, 4096, 6, 128, 2048
+        wt = (torch.randn(nl * 2 * D, hidden, device="cuda", generator=g) / 64).to(torch.bfloat16)
+        x = (torch.randn(T, hidden, device="cuda", generator=g) / 64).to(torch.bfloat16)
+        bufs = [(torch.empty(rows, D, dtype=torch.uint8, device="cuda"),
+                 torch.empty(rows, D, dtype=torch.uint8, device="cuda"),
+                 torch.empty(rows, device="cuda"), torch.empty(rows, device="cuda"))
+                for _ in range(nl)]
+        caches = [hs2.kv_cache(*b_) for b_ in bufs]
+        calls = [lambda: hs2.hs2_bridge_kv(x, T, hidden, wt, nl, D, hs2.HS2_KV_FP8_E4M3, caches,
+                                           1000)] * 2
+    for c in calls:
+        l2_flush()
+        c()
+        torch.cuda.synchronize()
+    st = hs2.hs2_last_device_status()
+    print(json.dumps({"profile_case": name, "what": PROFILE_CASES[name], "status": st}), flush=True)
+    if st != 0:
+        raise SystemExit(1)
 
 
 def measured_tensor_peak():
@@ -652,6 +735,7 @@ def run_hs2(args, world, rank, local):
         c.record(stream)
     torch.cuda.synchronize()
     e2e_ms = [a.elapsed_time(c) for a, c in e2e_ev]
+    phases = fused_phases(torch, hs2, l2_flush, lambda: step(qs), 2 * B * L * D * 2 + B * T * H * D * 2)
 
     def agg(xs):
         return max_over_ranks(float(np.median(xs)), world, "cuda")
@@ -725,6 +809,7 @@ def run_hs2(args, world, rank, local):
                          "frac": sparse_bytes / (sparse * 1e-3) / 1e9 / peak},
         "full_ms": full,
         "instrumented_ms_per_step": inst,
+        "fused_phases": phases,
         "clocks": clk,
         "cpu_baseline": cpu,
         "bridge": bridge,
@@ -733,6 +818,42 @@ def run_hs2(args, world, rank, local):
         "configs": others,
     }
     print(json.dumps(line), flush=True)
+
+
+def fused_phases(torch, hs2, l2_flush, call, stream_bytes, reps=5):
+    """Where the fused kernel's time goes, from the global-timer stamps its CTAs
+    write when enabled (outside every timed region; L2 flushed before each
+    call).  Times in us from the first CTA's start, medians over `reps` calls:
+    when the last CTA finished its partial pass (every K/V tile streamed),
+    passed each group barrier, finished the score pass and finished; and the
+    partial pass's achieved bandwidth: K and V once plus the queries over
+    first start -> last partial done."""
+    n = 1024
+    buf = torch.zeros(n * hs2.HS2_PHASES, dtype=torch.int64, device="cuda")
+    rows = []
+    try:
+        hs2.hs2_set_phase_stamps(buf, n)
+        for _ in range(reps):
+            buf.zero_()
+            l2_flush()
+            call()
+            torch.cuda.synchronize()
+            st = buf.view(n, hs2.HS2_PHASES).cpu().numpy()
+            st = st[st[:, 0] > 0]
+            t0 = st[:, 0].min()
+            rows.append([(st[:, k].max() - t0) / 1e3 if (st[:, k] > 0).all() else float("nan")
+                         for k in range(7)])
+    finally:
+        hs2.hs2_set_phase_stamps(None)
+    med = np.nanmedian(np.array(rows), axis=0)
+    names = ["start_spread", "partial_done", "barrier1", "score_done", "barrier2", "barrier3", "end"]
+    out = {k: (float(v) if np.isfinite(v) else None) for k, v in zip(names, med)}
+    out["unit"] = "us from the first CTA's start (latest CTA per phase)"
+    if out["partial_done"]:
+        peak, _ = measured_peaks()
+        out["stream_gbs"] = stream_bytes / (out["partial_done"] * 1e-6) / 1e9
+        out["stream_frac"] = out["stream_gbs"] / peak
+    return out
 
 
 def run_section(args):
@@ -767,7 +888,9 @@ def run_section(args):
 def main():
     args = parse()
     world, rank, local = dist_setup()
-    if args.only:
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+    elif args.only:
         run_section(args)
     elif args.impl == "reference":
         run_reference(args, world, rank)

@@ -355,6 +355,26 @@ HS2_API hs2_status hs2_set_stage_events(void* begin_event, void* end_event);
  */
 HS2_API hs2_status hs2_set_fault_injection(unsigned extra_arrivals, unsigned long long wait_limit_ns);
 
+/*
+ * Phase timestamps of the fused full-attention kernel (the decode path of
+ * hs2_full_attn_select: head_dim 128, 32 query rows per group), for tracing
+ * where its time goes.  While `stamps` is set, every CTA b < max_ctas of that
+ * kernel writes HS2_PHASES values of the GPU's nanosecond global timer to
+ * stamps[b * HS2_PHASES + i]:
+ *   0 CTA start, 1 its partial pass done (every K/V tile streamed and its
+ *   partial written), 2 first group barrier passed, 3 score pass and output
+ *   merge done, 4 second group barrier passed, 5 third group barrier passed
+ *   (selection), 6 CTA done; the eighth value is not written.
+ * A stamp a CTA does not reach (a phase the call skips) is left as it was.
+ *   stamps: device buffer of max_ctas * HS2_PHASES uint64 values, owned by the
+ *     caller; NULL (the default) turns the stamps off.
+ * The setting applies to the full-attention calls made afterwards on this host
+ * thread.  Returns HS2_ERR_INVALID_ARG for a non-null stamps with max_ctas < 1
+ * or a buffer not 8-byte aligned.  Nothing is enqueued by this call.
+ */
+#define HS2_PHASES 8
+HS2_API hs2_status hs2_set_phase_stamps(unsigned long long* stamps, int max_ctas);
+
 /* Library ABI version: 100 * major + minor. */
 HS2_API int hs2_version(void);
 

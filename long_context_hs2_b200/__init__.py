@@ -28,7 +28,10 @@ EXPORTED = ("hs2_bridge_kv", "hs2_full_attn_select_workspace", "hs2_full_attn_se
             "hs2_status_string", "hs2_version", "hs2_set_stage_events",
             "hs2_set_fault_injection", "hs2_full_attn_select_blocks", "hs2_cp_workspace",
             "hs2_cp_attn_partial", "hs2_cp_lse_combine", "hs2_cp_rescale", "hs2_cp_select_local",
-            "hs2_cp_merge_select")
+            "hs2_cp_merge_select", "hs2_set_phase_stamps")
+
+# Global-timer stamps per CTA written by the fused full-attention kernel when enabled.
+HS2_PHASES = 8
 
 # Size of the scratch area built into the library for hs2_full_attn_select_noalloc.
 HS2_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -94,6 +97,8 @@ def load_library(path: str = LIB_PATH):
     lib.hs2_set_stage_events.restype = i32
     lib.hs2_set_fault_injection.restype = i32
     lib.hs2_set_fault_injection.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
+    lib.hs2_set_phase_stamps.restype = i32
+    lib.hs2_set_phase_stamps.argtypes = [ctypes.c_void_p, ctypes.c_int]
     lib.hs2_set_stage_events.argtypes = [P, P]
     lib.hs2_sparse_attn.restype = i32
     lib.hs2_sparse_attn.argtypes = [P, KV, i32, i32, i64, i32, i32, ctypes.c_float, P, P, i32, i32,
@@ -205,6 +210,14 @@ def hs2_set_stage_events(begin=None, end=None):
             return e
         return e.cuda_event
     _check("hs2_set_stage_events", load_library().hs2_set_stage_events(handle(begin), handle(end)))
+
+
+def hs2_set_phase_stamps(stamps=None, max_ctas: int = 0):
+    """Tracing: the fused full-attention kernel writes HS2_PHASES global-timer
+    stamps per CTA into `stamps` (a device uint64/int64 buffer of max_ctas *
+    HS2_PHASES values); None turns them off."""
+    _check("hs2_set_phase_stamps",
+           load_library().hs2_set_phase_stamps(_ptr(stamps), int(max_ctas) if stamps is not None else 0))
 
 
 def hs2_set_fault_injection(extra_arrivals: int = 0, wait_limit_ns: int = 0):

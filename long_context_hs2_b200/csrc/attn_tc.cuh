@@ -288,6 +288,9 @@ __device__ __forceinline__ void tc_partial_setup(uint8_t* smem) {
 // columns each beside the 32 of O^T: all 512 columns).
 constexpr int kTcRetainTiles = 15;
 
+// Phase stamps per CTA of the fused kernel (tracing).
+constexpr int kPhases = 8;
+
 
 // The partial pass of one (group, split) work item: every role's work, with
 // the barriers of tc_partial_setup initialised and the TMEM columns at `tmem`
@@ -786,6 +789,12 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   uint64_t* k2_full = s2_empty + 2;    // [2], E4M3 only
   uint64_t* k2_free = k2_full + 2;     // [2]
 
+  // phase k of this CTA reached: one global-timer stamp (tracing; off when null)
+  auto stamp = [&](int k) {
+    if (p.phase_stamps && threadIdx.x == 0 && (int)blockIdx.x < p.phase_ctas)
+      p.phase_stamps[blockIdx.x * kPhases + k] = globaltimer();
+  };
+  stamp(0);
   pdl_launch_dependents();  // a following sparse layer may place its CTAs on idle SMs
   tc_partial_setup<N, FP8>(smem);
   if (threadIdx.x == 0) {
@@ -835,10 +844,13 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     }
   };
   tc_fence_before();
+  if (p.phase_stamps) __syncthreads();  // (uniform) every role's part of the pass is done
+  stamp(1);
   if (!group_arrive_wait(gsync, target, p.wait_limit_ns)) {  // the group's partials are out
     give_up();
     return;
   }
+  stamp(2);
   tc_fence_after();
 
   // --------------------------------------------------------- score pass
@@ -1093,6 +1105,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   }
   tc_fence_before();
   __syncthreads();
+  stamp(3);
 
   // ------------------------------------------ selection (whole group)
   // The k-th largest score pattern tau, as in select_topk_kernel, in two group
@@ -1145,6 +1158,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       give_up();
       return;
     }
+    stamp(4);
 #pragma unroll 1
     for (int q = 0; q < G; ++q)
       if (active(q)) {
@@ -1193,6 +1207,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       give_up();
       return;
     }
+    stamp(5);
 #pragma unroll 1
     for (int q = 0; q < G; ++q)
       if (active(q)) {
@@ -1354,6 +1369,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   }
   tc_fence_before();
   __syncthreads();
+  stamp(6);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

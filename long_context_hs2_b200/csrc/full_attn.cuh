@@ -53,6 +53,9 @@ struct FullAttnParams {
   // group's CTA count (non-zero only under fault injection)
   unsigned long long wait_limit_ns;
   unsigned barrier_extra;
+  // fused kernel: kPhases global-timer stamps per CTA b < phase_ctas (null: off)
+  unsigned long long* phase_stamps;
+  int phase_ctas;
   // query t sits at local key position qpos0 + t (L - T when the cache holds
   // the whole context; with a context-parallel slice, the queries' position
   // relative to the slice's first key, which may exceed L)

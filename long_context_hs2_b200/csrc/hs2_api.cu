@@ -78,6 +78,8 @@ thread_local cudaEvent_t t_stage_begin = nullptr, t_stage_end = nullptr;
 
 // ------------------------------------------------- fault injection --
 constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;
+thread_local unsigned long long* t_phase_stamps = nullptr;
+thread_local int t_phase_ctas = 0;
 thread_local unsigned t_barrier_extra = 0;
 thread_local unsigned long long t_wait_limit_ns = kDefaultWaitLimitNs;
 
@@ -435,6 +437,15 @@ hs2_status hs2_set_fault_injection(unsigned extra_arrivals, unsigned long long w
   return HS2_OK;
 }
 
+static_assert(HS2_PHASES == hs2::kPhases, "phase stamps per CTA");
+
+hs2_status hs2_set_phase_stamps(unsigned long long* stamps, int max_ctas) {
+  if (stamps && (max_ctas < 1 || ((uintptr_t)stamps & 7u) != 0)) return HS2_ERR_INVALID_ARG;
+  t_phase_stamps = stamps;
+  t_phase_ctas = stamps ? max_ctas : 0;
+  return HS2_OK;
+}
+
 hs2_status hs2_set_stage_events(void* begin_event, void* end_event) {
   if ((begin_event == nullptr) != (end_event == nullptr)) return HS2_ERR_INVALID_ARG;
   t_stage_begin = static_cast<cudaEvent_t>(begin_event);
@@ -539,6 +550,8 @@ hs2_status setup_full(const void* Q, const hs2_kv_cache* kv, int B, int T, int64
   fp.topk = topk;
   fp.slots = topk + window;
   fp.fuse_select = 0;
+  fp.phase_stamps = t_phase_stamps;
+  fp.phase_ctas = t_phase_ctas;
   fp.wait_limit_ns = t_wait_limit_ns;
   fp.barrier_extra = t_barrier_extra;
   fp.qpos0 = L - T;

@@ -280,6 +280,37 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
   for (int b = threadIdx.x; b < 2048; b += kSelThreads) h2[b] = 0u;
   for (int b = threadIdx.x; b < 512; b += kSelThreads) h3[b] = 0u;
   __syncthreads();
+  // fn(v) for every candidate of the segment, in no particular order.  From
+  // global memory (rows too long for shared memory) with 16-byte loads,
+  // kBatch of them in flight per thread: one 4-byte load per thread at a time
+  // leaves a row pass bound by memory latency, not bandwidth.
+  const bool vec = !SMEM && (((uintptr_t)src) & 15u) == 0;
+  auto each = [&](auto&& fn) {
+    if (vec) {
+      constexpr int kBatch = 4;
+      const uint4* s4 = reinterpret_cast<const uint4*>(src);
+      const int n4 = n >> 2;
+      for (int j0 = threadIdx.x; j0 < n4; j0 += kBatch * kSelThreads) {
+        uint4 v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int j = j0 + u * kSelThreads;
+          v[u] = j < n4 ? s4[j] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          if (j0 + u * kSelThreads < n4) {
+            fn(v[u].x);
+            fn(v[u].y);
+            fn(v[u].z);
+            fn(v[u].w);
+          }
+      }
+      for (int j = 4 * n4 + threadIdx.x; j < n; j += kSelThreads) fn(src[j]);
+    } else {
+      for (int j = threadIdx.x; j < n; j += kSelThreads) fn(src[j]);
+    }
+  };
 
   int need = p.topk;
   unsigned prefix = 0;
@@ -293,13 +324,12 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
     // shared-memory atomics); after a cluster barrier each CTA copies it.
     const uint32_t h2_0 = cs > 1 ? sel_mapa(smem_u32(h2), 0) : 0u;
     if (cs > 1) sel_cluster_sync();  // rank 0's histograms are cleared
-    for (int j = threadIdx.x; j < n; j += kSelThreads) {
-      const unsigned v = src[j];
+    each([&](unsigned v) {
       if ((v >> 20) == prefix) {
         if (cs > 1) red_dsmem_add_u32(h2_0 + ((v >> 9) & 2047u) * 4, 1u);
         else atomicAdd(&h2[(v >> 9) & 2047u], 1u);
       }
-    }
+    });
     const unsigned* h = h2;
     if (cs > 1) {
       sel_cluster_sync();
@@ -312,13 +342,12 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
     need = res[1];
     // level 3: bits [8:0] among elements with bits[30:9] == prefix
     const uint32_t h3_0 = cs > 1 ? sel_mapa(smem_u32(h3), 0) : 0u;
-    for (int j = threadIdx.x; j < n; j += kSelThreads) {
-      const unsigned v = src[j];
+    each([&](unsigned v) {
       if ((v >> 9) == prefix) {
         if (cs > 1) red_dsmem_add_u32(h3_0 + (v & 511u) * 4, 1u);
         else atomicAdd(&h3[v & 511u], 1u);
       }
-    }
+    });
     h = h3;
     if (cs > 1) {
       sel_cluster_sync();
@@ -338,12 +367,21 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
   const int wseg = (n + kSelThreads / 32 - 1) / (kSelThreads / 32);
   const int w0 = min(n, warp * wseg), w1 = min(n, w0 + wseg);
   int n_gt = 0, n_eq = 0;
+  constexpr int kChunks = 4;  // 32-candidate chunks loaded together (in order afterwards)
   if (p.topk > 0) {
-    for (int base = w0; base < w1; base += 32) {
-      const int j = base + lane;
-      const unsigned v = j < w1 ? src[j] : 0u;
-      n_gt += __popc(__ballot_sync(0xffffffffu, j < w1 && v > tau));
-      n_eq += __popc(__ballot_sync(0xffffffffu, j < w1 && v == tau));
+    for (int base = w0; base < w1; base += 32 * kChunks) {
+      unsigned v[kChunks];
+#pragma unroll
+      for (int u = 0; u < kChunks; ++u) {
+        const int j = base + 32 * u + lane;
+        v[u] = j < w1 ? src[j] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kChunks; ++u) {
+        const int j = base + 32 * u + lane;
+        n_gt += __popc(__ballot_sync(0xffffffffu, j < w1 && v[u] > tau));
+        n_eq += __popc(__ballot_sync(0xffffffffu, j < w1 && v[u] == tau));
+      }
     }
   }
   if (lane == 0) {
@@ -387,24 +425,33 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
   if (p.topk > 0) {
     int pos = gt_before + min(eq_before, need);
     int eq_rank = eq_before;
-    for (int base = w0; base < w1; base += 32) {
-      const int j = base + lane;
-      const unsigned v = j < w1 ? src[j] : 0u;
-      const bool gt = j < w1 && v > tau;
-      const bool eq = j < w1 && v == tau;
-      const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-      const int my_eq_rank = eq_rank + __popc(eqm & ((1u << lane) - 1u));
-      const bool sel = gt || (eq && my_eq_rank < need);
-      const unsigned selm = __ballot_sync(0xffffffffu, sel);
-      if (sel) {
-        const int o = pos + __popc(selm & ((1u << lane) - 1u));
-        if (o < p.topk) {
-          out[o] = (int32_t)(s0 + j + p.key_off);
-          if (p.cp) p.cand_score[row * p.slots + o] = __uint_as_float(v);
-        }
+    for (int base = w0; base < w1; base += 32 * kChunks) {
+      unsigned vc[kChunks];
+#pragma unroll
+      for (int u = 0; u < kChunks; ++u) {
+        const int j = base + 32 * u + lane;
+        vc[u] = j < w1 ? src[j] : 0u;
       }
-      pos += __popc(selm);
-      eq_rank += __popc(eqm);
+#pragma unroll
+      for (int u = 0; u < kChunks; ++u) {
+        const int j = base + 32 * u + lane;
+        const unsigned v = vc[u];
+        const bool gt = j < w1 && v > tau;
+        const bool eq = j < w1 && v == tau;
+        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+        const int my_eq_rank = eq_rank + __popc(eqm & ((1u << lane) - 1u));
+        const bool sel = gt || (eq && my_eq_rank < need);
+        const unsigned selm = __ballot_sync(0xffffffffu, sel);
+        if (sel) {
+          const int o = pos + __popc(selm & ((1u << lane) - 1u));
+          if (o < p.topk) {
+            out[o] = (int32_t)(s0 + j + p.key_off);
+            if (p.cp) p.cand_score[row * p.slots + o] = __uint_as_float(v);
+          }
+        }
+        pos += __popc(selm);
+        eq_rank += __popc(eqm);
+      }
     }
     if (rank == (uint32_t)(cs - 1) && warp == kSelThreads / 32 - 1 && lane == 0 && pos != p.topk)
       raise_status(kStatusBadIndex);

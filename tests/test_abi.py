@@ -108,6 +108,13 @@ def test_fault_injection_setter(lib):
     assert lib.hs2_set_fault_injection(0, 0) == 0
 
 
+def test_phase_stamps_setter(lib):
+    # the setter only records the buffer for later calls: it checks its arguments
+    assert lib.hs2_set_phase_stamps(ctypes.c_void_p(4096), 0) == 1
+    assert lib.hs2_set_phase_stamps(ctypes.c_void_p(4100), 8) == 1
+    assert lib.hs2_set_phase_stamps(None, 0) == 0
+
+
 def test_stage_events_pairing(lib):
     assert lib.hs2_set_stage_events(ctypes.c_void_p(16), None) == 1
     assert lib.hs2_set_stage_events(None, ctypes.c_void_p(16)) == 1
