@@ -63,6 +63,8 @@ PROFILE_CASES = {
     "decode_fp8": "hs2_full_attn_select on the 4 x 256K E4M3 decode workload",
     "chunk_small": "hs2_full_attn_select on a 512-query chunk over 128K E4M3 tokens",
     "sparse_chunk": "hs2_sparse_attn on a 1024-query chunk over 256K E4M3 tokens",
+    "sparse_decode": "hs2_sparse_attn on the 8 x 32K bf16 decode workload",
+    "bridge_131k": "hs2_bridge_kv of 131072 tokens into 6 layers' bf16 caches",
     "bridge_append": "hs2_bridge_kv of 64 tokens into 6 layers' E4M3 caches",
 }
 
@@ -116,6 +118,18 @@ def run_profile_case(name):
     elif name == "sparse_chunk":
         full, sparse = attn("chunk_fp8_1m", T=1024, L=262144)
         calls = [full, sparse, sparse]
+    elif name == "sparse_decode":
+        full, sparse = attn("decode_bf16_32k")
+        calls = [full, sparse, sparse]
+    elif name == "bridge_131k":
+        T, hidden, nl, D = 131072, 4096, 6, 128
+        wt = (torch.randn(nl * 2 * D, hidden, device="cuda", generator=g) / 64).to(torch.bfloat16)
+        x = (torch.randn(T, hidden, device="cuda", generator=g) / 64).to(torch.bfloat16)
+        bufs = [(torch.empty(T, D, dtype=torch.bfloat16, device="cuda"),
+                 torch.empty(T, D, dtype=torch.bfloat16, device="cuda"), None, None)
+                for _ in range(nl)]
+        caches = [hs2.kv_cache(*b_) for b_ in bufs]
+        calls = [lambda: hs2.hs2_bridge_kv(x, T, hidden, wt, nl, D, hs2.HS2_KV_BF16, caches, 0)] * 2
     else:  # bridge_append
         T, hidden, nl, D, rows = 64, 4096, 6, 128, 2048
         wt = (torch.randn(nl * 2 * D, hidden, device="cuda", generator=g) / 64).to(torch.bfloat16)

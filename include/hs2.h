@@ -362,9 +362,10 @@ HS2_API hs2_status hs2_set_fault_injection(unsigned extra_arrivals, unsigned lon
  * kernel writes HS2_PHASES values of the GPU's nanosecond global timer to
  * stamps[b * HS2_PHASES + i]:
  *   0 CTA start, 1 its partial pass done (every K/V tile streamed and its
- *   partial written), 2 first group barrier passed, 3 score pass and output
- *   merge done, 4 second group barrier passed, 5 third group barrier passed
- *   (selection), 6 CTA done; the eighth value is not written.
+ *   partial written), 2 first group barrier passed, 3 its score pass done
+ *   (candidate scores and histogram counts issued), 4 second group barrier
+ *   passed, 5 third group barrier passed (selection), 6 CTA done; the eighth
+ *   value is not written.
  * A stamp a CTA does not reach (a phase the call skips) is left as it was.
  *   stamps: device buffer of max_ctas * HS2_PHASES uint64 values, owned by the
  *     caller; NULL (the default) turns the stamps off.

@@ -790,8 +790,11 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   uint64_t* k2_free = k2_full + 2;     // [2]
 
   // phase k of this CTA reached: one global-timer stamp (tracing; off when null)
-  auto stamp = [&](int k) {
-    if (p.phase_stamps && threadIdx.x == 0 && (int)blockIdx.x < p.phase_ctas)
+  // (written by thread `by` of the CTA, at a point that thread reaches only
+  // once the phase is done: a timer read right after a block barrier may be
+  // scheduled before it)
+  auto stamp = [&](int k, int by = 0) {
+    if (p.phase_stamps && threadIdx.x == by && (int)blockIdx.x < p.phase_ctas)
       p.phase_stamps[blockIdx.x * kPhases + k] = globaltimer();
   };
   stamp(0);
@@ -843,9 +846,8 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       tmem_dealloc(tmem, kTmemCols);
     }
   };
+  stamp(1, 64);  // the first softmax thread has written its rows' partials
   tc_fence_before();
-  if (p.phase_stamps) __syncthreads();  // (uniform) every role's part of the pass is done
-  stamp(1);
   if (!group_arrive_wait(gsync, target, p.wait_limit_ns)) {  // the group's partials are out
     give_up();
     return;
@@ -1059,6 +1061,7 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         if (cnt && t < p.T)
           atomicAdd(&p.hist[((long long)b * p.T + t) * kHistBins + (u % kHistBins)], cnt);
       }
+      stamp(3, 64);  // the score warps' candidate scores and histogram counts are out
     } else {
       // ---- merge warps 6-9: output row r of the group is merged by the CTA of
       //      split r mod ns; thread d owns element d
@@ -1105,7 +1108,6 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   }
   tc_fence_before();
   __syncthreads();
-  stamp(3);
 
   // ------------------------------------------ selection (whole group)
   // The k-th largest score pattern tau, as in select_topk_kernel, in two group

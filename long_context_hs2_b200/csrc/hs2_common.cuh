@@ -22,9 +22,12 @@ constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 __device__ __forceinline__ void raise_status(unsigned bits) { atomicOr(&g_status, bits); }
 
+// The GPU's nanosecond timer.  The memory clobber keeps the read in program
+// order with memory operations and barriers (a timestamp taken after a block
+// barrier must not be scheduled before it).
 __device__ __forceinline__ unsigned long long globaltimer() {
   unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t) : : "memory");
   return t;
 }
 
