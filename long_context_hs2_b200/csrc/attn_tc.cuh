@@ -229,12 +229,15 @@ __device__ __forceinline__ void tc_issue_pv(uint32_t tmem_d, uint32_t v_addr, ui
 }
 
 // Partial kernel: warps 0 (TMA), 1 (MMA) and 8 softmax warps 2-9 (plus, for
-// an E4M3 cache, K converter warps 10-11 and V converter warps 12-13).
+// an E4M3 cache, K converter warps 10-12 and V converter warps 13-15).
 // Softmax warp w reads TMEM lane quarter w%4 (keys, or d for O^T) and the
 // column half (w-2)/4 of the N rows, so two warps share each scheduler and
 // each thread handles one key x N/2 rows per tile.
 constexpr int kTcSoftmax = 256;
-constexpr int kTcConvert = 64;  // threads per converted tensor (K or V)
+// Three converter warps per tensor: with two, the E4M3 -> f16 conversion set the
+// per-tile time (measured on B200: 256K decode call 0.215 -> 0.207 ms, 1M chunk
+// 238 -> 226 ms with three).
+constexpr int kTcConvert = 96;  // threads per converted tensor (K or V)
 __host__ __device__ constexpr int tc_partial_threads(bool fp8) {
   return 64 + kTcSoftmax + (fp8 ? 2 * kTcConvert : 0);
 }
@@ -526,27 +529,102 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
         for (int c = 0; c < NC; c += 16) tmem_ld16(s_addr + c, xs + (c % (kHold ? NC : 16)));
         tmem_ld_wait();
       }
-      // sweep 1: does any logit exceed its row's reference by more than 2^8?
-      bool need = false;
+      // p = 2^(x - m_ref), row sums, P^T (bf16, or f16 times the value scale for
+      // an E4M3 cache) for the PV product; RETAIN: p replaces the logits in the
+      // tile's TMEM block, with the tile's reference kept.  With `guard`, a logit
+      // above its row's reference by more than 2^8 counts as 0 and is reported
+      // (the tile is then redone after a rescale); undo: subtract the same
+      // guarded values from the row sums again.
+      uint8_t* pt = p_base + (n % NP) * SM::kPBytes;
+      auto sweep = [&](bool guard, bool undo) {
+        bool over_any = false;
 #pragma unroll
-      for (int c = 0; c < NC; c += 16) {
-        if (!kHold) {
-          tmem_ld16(s_addr + c, xs);
-          tmem_ld_wait();
+        for (int c = 0; c < NC; c += 16) {
+          float lv[16], pk[16];
+          if (!kHold) tmem_ld16(s_addr + c, xs);
+          if (RETAIN) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) lv[i] = lreg[(c + i) % (RETAIN ? NC : 1)];
+          } else {
+            tmem_ld16(tmem + lane_base + 3 * N + c0 + c, lv);
+          }
+          if (!kHold || !RETAIN) tmem_ld_wait();
+          const float* x = xs + (kHold ? c : 0);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int col = c0 + c + i;
+            const bool ok = full_tile || vis[(c + i) / kH];
+            const float mr = m_ref[col];
+            const float xl = x[i] * sl;
+            const bool over = guard && ok && xl > mr + kRescaleAbove;
+            over_any |= over;
+            const float pr = (ok && !over && mr != kNegInf) ? fast_exp2(xl - mr) : 0.f;
+            pk[i] = pr;
+            lv[i] = undo ? lv[i] - pr : lv[i] + pr;
+            if (kPMN || undo) continue;
+            if (FP8)
+              *reinterpret_cast<__half*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
+                  __float2half_rn(pr * vsc);
+            else
+              *reinterpret_cast<__nv_bfloat16*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
+                  __float2bfloat16_rn(pr);
+          }
+          if (kPMN && !undo) {  // this key's 16 rows c0+c .. c0+c+15: two packed 16-byte chunks
+            uint32_t w[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              w[u] = FP8 ? pack_f16(pk[2 * u] * vsc, pk[2 * u + 1] * vsc)
+                         : pack_bf16(pk[2 * u], pk[2 * u + 1]);
+            uint8_t* prow = pmn_row + (n % NP) * SM::kPBytes;
+            const int ch = c >> 3;
+            *reinterpret_cast<uint4*>(prow + ((ch ^ (keyrow & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(prow + (((ch + 1) ^ (keyrow & 7)) << 4)) =
+                make_uint4(w[4], w[5], w[6], w[7]);
+          }
+          if (RETAIN) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) lreg[(c + i) % (RETAIN ? NC : 1)] = lv[i];
+            tmem_st16(s_addr + c, pk);
+          } else {
+            tmem_st16(tmem + lane_base + 3 * N + c0 + c, lv);
+          }
         }
+        return over_any;
+      };
+      // Wide rows (kOne: not held in registers) take one sweep with the current
+      // references and redo the tile only when one must be raised (rare after
+      // the first tiles); 16-column rows check first (sweep 1), then sweep.
+      constexpr bool kOne = !kHold && !RETAIN;
+      bool need = false;
+      if (!kOne) {
+        // sweep 1: does any logit exceed its row's reference by more than 2^8?
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const bool ok = full_tile || vis[(c + i) / kH];
-          need |= ok && xs[(kHold ? c : 0) + i] * sl > m_ref[c0 + c + i] + kRescaleAbove;
+        for (int c = 0; c < NC; c += 16) {
+          if (!kHold) {
+            tmem_ld16(s_addr + c, xs);
+            tmem_ld_wait();
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const bool ok = full_tile || vis[(c + i) / kH];
+            need |= ok && xs[(kHold ? c : 0) + i] * sl > m_ref[c0 + c + i] + kRescaleAbove;
+          }
         }
       }
       if (n >= NP) {  // the P^T buffer of this tile is free once PV(n - NP) is done
         failed |= !mbar_wait(&pv_done[n % NP], ((n - NP) / NP) & 1);
         tc_fence_after();
       }
+      if (kOne) need = sweep(true, false);
       const bool any_need = softmax_any<kTcSoftmax>(need);
       if (softmax_any<kTcSoftmax>(failed)) break;
       if (any_need) {
+        if (kOne) {  // the row sums lose this tile's guarded values again
+          tmem_st_wait();
+          sweep(true, true);
+          tmem_st_wait();
+        }
         // new reference: column max of this tile's logits (and the old reference)
 #pragma unroll
         for (int c = 0; c < NC; c += 16) {
@@ -597,60 +675,9 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
         }
         tmem_st_wait();  // the rescaled row sums are read back below
       }
-      // sweep 2: p = 2^(x - m_ref), row sums, P^T (bf16, or f16 times the
-      // value scale for an E4M3 cache) for the PV product; RETAIN: p replaces
-      // the logits in the tile's TMEM block, with the tile's reference kept
-      uint8_t* pt = p_base + (n % NP) * SM::kPBytes;
       if (RETAIN && st < N)
         reinterpret_cast<float*>(smem + SM::kMhistOff)[n * N + st] = m_ref[st];
-#pragma unroll
-      for (int c = 0; c < NC; c += 16) {
-        float lv[16], pk[16];
-        if (!kHold) tmem_ld16(s_addr + c, xs);
-        if (RETAIN) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) lv[i] = lreg[(c + i) % (RETAIN ? NC : 1)];
-        } else {
-          tmem_ld16(tmem + lane_base + 3 * N + c0 + c, lv);
-        }
-        if (!kHold || !RETAIN) tmem_ld_wait();
-        const float* x = xs + (kHold ? c : 0);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int col = c0 + c + i;
-          const bool ok = full_tile || vis[(c + i) / kH];
-          const float mr = m_ref[col];
-          const float pr = (ok && mr != kNegInf) ? fast_exp2(x[i] * sl - mr) : 0.f;
-          pk[i] = pr;
-          lv[i] += pr;
-          if (kPMN) continue;
-          if (FP8)
-            *reinterpret_cast<__half*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
-                __float2half_rn(pr * vsc);
-          else
-            *reinterpret_cast<__nv_bfloat16*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
-                __float2bfloat16_rn(pr);
-        }
-        if (kPMN) {  // this key's 16 rows c0+c .. c0+c+15: two packed 16-byte chunks
-          uint32_t w[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) w[u] = FP8 ? pack_f16(pk[2 * u] * vsc, pk[2 * u + 1] * vsc)
-                                                 : pack_bf16(pk[2 * u], pk[2 * u + 1]);
-          uint8_t* prow = pmn_row + (n % NP) * SM::kPBytes;
-          const int ch = c >> 3;
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (keyrow & 7)) << 4)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
-          *reinterpret_cast<uint4*>(prow + (((ch + 1) ^ (keyrow & 7)) << 4)) =
-              make_uint4(w[4], w[5], w[6], w[7]);
-        }
-        if (RETAIN) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) lreg[(c + i) % (RETAIN ? NC : 1)] = lv[i];
-          tmem_st16(s_addr + c, pk);
-        } else {
-          tmem_st16(tmem + lane_base + 3 * N + c0 + c, lv);
-        }
-      }
+      if (!kOne || any_need) sweep(false, false);
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
@@ -803,12 +830,12 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S2; ++s) {
       mbar_init(&kv2_full[s], 1);
-      mbar_init(&kv2_empty[s], FP8 ? 4 : 1);
+      mbar_init(&kv2_empty[s], FP8 ? 2 * kTcConvert / 32 : 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s2_full[i], 1);
       mbar_init(&s2_empty[i], 4);
-      mbar_init(&k2_full[i], 4);
+      mbar_init(&k2_full[i], 2 * kTcConvert / 32);
       mbar_init(&k2_free[i], 1);
     }
     fence_mbar_init();
@@ -899,14 +926,16 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       }
     }
   } else if (FP8 && warp >= 2 + kTcSoftmax / 32) {
-    // E4M3 -> f16: converter warp 10 + i takes key rows 32i .. 32i+31 of a tile
-    const int i = warp - (2 + kTcSoftmax / 32);
-    if (i < 4 && !RETAIN)
+    // E4M3 -> f16: every converter warp (both the partial pass's K and V ones)
+    // converts its share of each K tile
+    const int ct = threadIdx.x - (64 + kTcSoftmax);
+    if (!RETAIN)
       for (int n = 0; n < n2; ++n) {
         const int s = n % S2, bb = n & 1;
         if (!mbar_wait(&kv2_full[s], (n / S2) & 1)) break;
         if (n >= 2 && !mbar_wait(&k2_free[bb], ((n - 2) >> 1) & 1)) break;
-        fp8_rows_to_f16(smem + s * SM::kS2TileBytes, 32 * i, 32, lane, 32, k16 + bb * kTcTileBytes);
+        fp8_rows_to_f16(smem + s * SM::kS2TileBytes, 0, kTcKeys, ct, 2 * kTcConvert,
+                        k16 + bb * kTcTileBytes);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
