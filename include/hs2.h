@@ -266,6 +266,15 @@ HS2_API hs2_status hs2_cp_merge_select(const float* cand_score, const int32_t* c
  * outside [0, L) raise HS2_ERR_DEVICE through hs2_last_device_status and are
  * skipped.  A query with n_sel == 0 gets O = 0.
  * Supported: D in {64, 128}; H in {8, 16, 32}; slots <= 4096.
+ * Ordering: the kernel is launched with programmatic dependent launch and
+ * reads idx, n_sel and the K/V rows they name before waiting for the previous
+ * kernel of the stream to finish (so that, in a block of sparse layers, it
+ * gathers while the layer before it computes); after the wait it reads idx and
+ * n_sel again and gathers anew if they changed.  Q is read after the wait.  A
+ * kernel that precedes this call on the stream and itself lets dependent
+ * launches start early must therefore not write the cache rows it uses after
+ * doing so (this library's kernels never write the cache after letting a
+ * dependent start).
  */
 HS2_API hs2_status hs2_sparse_attn(const void* Q, const hs2_kv_cache* kv, int B, int T, int64_t L, int H,
                            int D, float scale, const int32_t* idx, const int32_t* n_sel,

@@ -120,7 +120,6 @@ __global__ void __launch_bounds__(kSpThreads) sparse_attn_kernel(const SparsePar
   // first cluster phase: this CTA runs (its merge inputs may be written once
   // the phase completes, just before the merge)
   if (cs > 1) cluster_arrive_relaxed();
-  pdl_wait();  // indices, counts and queries come from earlier kernels
   const uint32_t rank = cs > 1 ? cluster_ctarank() : 0u;
   const long long qrow = blockIdx.x / cs;  // b*T + t
   const int b = (int)(qrow / p.T);
@@ -132,16 +131,60 @@ __global__ void __launch_bounds__(kSpThreads) sparse_attn_kernel(const SparsePar
   const int lo = (int)rank * share;
   const int hi = min(lo + share, p.slots);
   const int tiles_max = (share + kSpTile - 1) / kSpTile;
-  // positions of the range, n_sel and the query rows (head h = row; rows >= H
-  // are zero) in one asynchronous round trip; slots past the range read as 0
-  // and are masked below
   int* nsel_s = pos_all + tiles_max * kSpTile;
-  if (threadIdx.x == 0) cp_async4(smem_u32(nsel_s), p.n_sel + qrow, 4);
-  for (int u = threadIdx.x; u < tiles_max * kSpTile; u += kSpThreads) {
-    const int slot = lo + u;
-    const bool in = slot < hi;
-    cp_async4(smem_u32(pos_all + u), in ? sel + slot : sel, in ? 4 : 0);
-  }
+  __shared__ int s_n_valid, s_redo;
+  // The range's positions (slots past the range read as 0) and n_sel: valid
+  // slots keep their position, the others -1 (out-of-range positions too,
+  // raising kStatusBadIndex when `report`).  All threads; ends with a barrier.
+  auto load_positions = [&](bool report) {
+    if (threadIdx.x == 0) cp_async4(smem_u32(nsel_s), p.n_sel + qrow, 4);
+    for (int u = threadIdx.x; u < tiles_max * kSpTile; u += kSpThreads) {
+      const int slot = lo + u;
+      const bool in = slot < hi;
+      cp_async4(smem_u32(pos_all + u), in ? sel + slot : sel, in ? 4 : 0);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    const int nv = max(0, min(max(0, min(*nsel_s, p.slots)), hi) - lo);
+    for (int u = threadIdx.x; u < tiles_max * kSpTile; u += kSpThreads) {
+      int ps = pos_all[u];
+      if (u >= nv) {
+        ps = -1;
+      } else if (ps < 0 || (long long)ps >= p.L) {
+        if (report) raise_status(kStatusBadIndex);
+        ps = -1;
+      }
+      pos_all[u] = ps;
+    }
+    if (threadIdx.x == 0) s_n_valid = nv;
+    __syncthreads();
+  };
+  // rows of tile k that hold a valid slot's group: whole 16-key groups
+  auto tile_rows = [&](int k, int nv) {
+    const int v = min(kSpTile, nv - k * kSpTile);
+    return (v + kSpGroup - 1) / kSpGroup * kSpGroup;
+  };
+  // prologue: fill kStages-1 ring slots (one commit group each)
+  auto gather_prologue = [&](int nv) {
+    const int mt = (nv + kSpTile - 1) / kSpTile;
+#pragma unroll
+    for (int s2 = 0; s2 < SM::kStages - 1; ++s2) {
+      if (s2 < mt)
+        sparse_gather_tile<D, FP8>(p, b, pos_all + s2 * kSpTile, tile_rows(s2, nv),
+                                   smem + s2 * SM::kStageBytes);
+      else
+        cp_async_commit();
+    }
+  };
+  // The positions and the first tiles' K/V rows are read before the wait on
+  // the previous kernel: in a block of sparse layers the indices were final
+  // before the previous layer began, and the gathers then overlap it.  After
+  // the wait the positions are read again; if any differs (indices rewritten
+  // by the previous kernel) the gathers are redone.
+  load_positions(false);
+  gather_prologue(s_n_valid);
+  pdl_wait();  // indices, counts and queries come from earlier kernels
   {
     constexpr int kChunks = D * 2 / 16;
     const uint32_t q_s = smem_u32(qs);
@@ -151,44 +194,50 @@ __global__ void __launch_bounds__(kSpThreads) sparse_attn_kernel(const SparsePar
       cp_async16(q_s + sw128_offset(r, ch * 16, SM::kRowsQ),
                  p.q + (qrow * p.H + (in ? r : 0)) * D + ch * 8, in ? 16 : 0);
     }
+    cp_async_commit();
   }
-  cp_async_commit();
-  cp_async_wait<0>();
+  {  // validate the positions read before the wait
+    const int nv0 = s_n_valid;
+    if (threadIdx.x == 0) s_redo = 0;
+    __syncthreads();
+    const int nsel_now = __ldcg(p.n_sel + qrow);
+    const int nv = max(0, min(max(0, min(nsel_now, p.slots)), hi) - lo);
+    bool differs = nv != nv0;
+    constexpr int kBatch = 8;  // independent loads in flight per thread
+    for (int u0 = threadIdx.x; u0 < nv0; u0 += kBatch * kSpThreads) {
+      int v[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        const int u = u0 + k * kSpThreads;
+        v[k] = u < nv0 ? __ldcg(sel + lo + u) : 0;
+      }
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        const int u = u0 + k * kSpThreads;
+        if (u < nv0) {
+          const int ps = (v[k] < 0 || (long long)v[k] >= p.L) ? -1 : v[k];
+          differs |= ps != pos_all[u];
+        }
+      }
+    }
+    if (differs) s_redo = 1;
+    __syncthreads();
+    if (s_redo) {  // (uniform) the gathers in flight land before the stages are refilled
+      cp_async_wait<0>();
+      __syncthreads();
+      load_positions(true);
+      gather_prologue(s_n_valid);
+    } else {
+      for (int u = threadIdx.x; u < nv0; u += kSpThreads)  // the status of bad positions
+        if (pos_all[u] < 0) raise_status(kStatusBadIndex);
+    }
+  }
+  cp_async_wait<0>();  // the query rows (and the prologue tiles, issued well before)
+  __syncthreads();
+  const int n_valid = s_n_valid;
+  const int my_tiles = (n_valid + kSpTile - 1) / kSpTile;
   const float* ksc = FP8 ? p.k_scale + (long long)b * p.L : nullptr;
   const float* vsc = FP8 ? p.v_scale + (long long)b * p.L : nullptr;
-
-  __syncthreads();
-  const int n = max(0, min(*nsel_s, p.slots));
-  const int end = min(hi, n);                  // valid slots: [lo, end)
-  const int n_valid = max(0, end - lo);
-  const int my_tiles = (n_valid + kSpTile - 1) / kSpTile;
-  // mask slots past n_sel or past the range; range-check the others
-  for (int u = threadIdx.x; u < my_tiles * kSpTile; u += kSpThreads) {
-    int ps = pos_all[u];
-    if (u >= n_valid) {
-      ps = -1;
-    } else if (ps < 0 || (long long)ps >= p.L) {
-      raise_status(kStatusBadIndex);
-      ps = -1;
-    }
-    pos_all[u] = ps;
-  }
-  __syncthreads();
-  // rows of tile k that hold a valid slot's group: whole 16-key groups
-  auto tile_rows = [&](int k) {
-    const int v = min(kSpTile, n_valid - k * kSpTile);
-    return (v + kSpGroup - 1) / kSpGroup * kSpGroup;
-  };
-
-  // prologue: fill kStages-1 ring slots
-#pragma unroll
-  for (int s = 0; s < SM::kStages - 1; ++s) {
-    if (s < my_tiles)
-      sparse_gather_tile<D, FP8>(p, b, pos_all + s * kSpTile, tile_rows(s),
-                                 smem + s * SM::kStageBytes);
-    else
-      cp_async_commit();
-  }
 
   WarpAttn<MT, D> st;
   st.init();
@@ -200,7 +249,7 @@ __global__ void __launch_bounds__(kSpThreads) sparse_attn_kernel(const SparsePar
     {  // refill the slot consumed in step k-1 (all threads passed the barrier ending it)
       const int kn = k + SM::kStages - 1;
       if (kn < my_tiles)
-        sparse_gather_tile<D, FP8>(p, b, pos_all + kn * kSpTile, tile_rows(kn),
+        sparse_gather_tile<D, FP8>(p, b, pos_all + kn * kSpTile, tile_rows(kn, n_valid),
                                    smem + (kn % SM::kStages) * SM::kStageBytes);
       else
         cp_async_commit();
@@ -209,7 +258,7 @@ __global__ void __launch_bounds__(kSpThreads) sparse_attn_kernel(const SparsePar
     __syncthreads();
     // this warp's 16-key group: skipped when it holds no valid slot (its rows
     // were not gathered)
-    if (warp * kSpGroup < tile_rows(k)) {
+    if (warp * kSpGroup < tile_rows(k, n_valid)) {
       const int s = k % SM::kStages;
       uint8_t* stage = smem + s * SM::kStageBytes;
       const int* pos = pos_all + k * kSpTile;
