@@ -241,7 +241,10 @@ constexpr int kTcConvert = 96;  // threads per converted tensor (K or V)
 __host__ __device__ constexpr int tc_partial_threads(bool fp8) {
   return 64 + kTcSoftmax + (fp8 ? 2 * kTcConvert : 0);
 }
-__host__ __device__ constexpr int tc_score_threads(bool fp8) { return fp8 ? 320 : 192; }
+// Score kernel: warps 0 (TMA), 1 (MMA), two groups of four score warps (2-5
+// take the even tiles, 6-9 the odd ones, each its own S^T buffer), and for an
+// E4M3 cache converter warps 10-13.
+__host__ __device__ constexpr int tc_score_threads(bool fp8) { return fp8 ? 448 : 320; }
 
 // Barrier initialisation and per-row state of the partial pass (all threads;
 // a block barrier must follow before the body runs).
@@ -298,9 +301,9 @@ constexpr int kPhases = 8;
 // The partial pass of one (group, split) work item: every role's work, with
 // the barriers of tc_partial_setup initialised and the TMEM columns at `tmem`
 // (4N; 512 when RETAIN).  TMEM layout: S^T double buffer at columns 0 and N,
-// O^T at 2N, per-key row sums at 3N; with RETAIN (N = 32, at most
-// kTcRetainTiles tiles) O^T at 0 and the S^T of tile n kept at N + n*N for a
-// later score pass, the row sums in registers.
+// O^T at 2N, per-key row sums at 3N (16-column rows: in registers); with
+// RETAIN (N = 32, at most kTcRetainTiles tiles) O^T at 0 and the S^T of tile n
+// kept at N + n*N for a later score pass.
 // Returns in every thread once its role is done (no trailing barrier).
 template <int N, int G, bool FP8, bool RETAIN = false>
 __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const CUtensorMap& vmap,
@@ -466,20 +469,23 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
     const int st = threadIdx.x - 64;         // softmax thread 0..255
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const int keyrow = wq * 32 + lane;       // row of S^T (key) / of O^T (d)
-    // P^T store address of (row c0 + c, this key): base + c*128 + xoff[(c0 + c) & 7]
+    // P^T store address of (row c0 + c, this key): base + c*128 + (the 16-byte
+    // chunk of this key's 8-key group, swizzled by the row) + 2 * (key & 7)
     // (K-major P^T); for 128-row groups P is stored MN-major instead: this
     // key's 128-byte row of the 64-row half c0/64, 16-byte chunks swizzled by key
     constexpr bool kPMN = tc_p_mn_major(N);
     uint8_t* p_base = smem + SM::kPOff + (keyrow >> 6) * (N * 128) + c0 * 128;
     uint8_t* pmn_row = smem + SM::kPOff + (c0 / 64) * (kTcKeys * 128) + keyrow * 128;
-    uint32_t xoff[8];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) xoff[m] = ((((keyrow & 63) >> 3) ^ m) << 4) + (keyrow & 7) * 2;
+    const uint32_t kchunk = (uint32_t)(keyrow & 63) >> 3;  // this key's 16-byte chunk of a row
+    const uint32_t kpair = (uint32_t)(keyrow & 6) * 2;     // its lane pair's byte in the chunk
     bool failed = false;
-    float lreg[RETAIN ? NC : 1];  // RETAIN: this key's row sums in registers
+    // this key's row sums: in registers for 16-column rows, else in TMEM at 3N
+    constexpr bool kLReg = NC <= 16;
+    static_assert(!RETAIN || kLReg, "a retaining pass keeps the row sums in registers");
+    float lreg[kLReg ? NC : 1];
 #pragma unroll
-    for (int i = 0; i < (RETAIN ? NC : 1); ++i) lreg[i] = 0.f;
-    if (!RETAIN) {  // TMEM is undefined at allocation: clear this thread's row sums
+    for (int i = 0; i < (kLReg ? NC : 1); ++i) lreg[i] = 0.f;
+    if (!kLReg) {  // TMEM is undefined at allocation: clear this thread's row sums
       float z[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) z[i] = 0.f;
@@ -542,13 +548,13 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
         for (int c = 0; c < NC; c += 16) {
           float lv[16], pk[16];
           if (!kHold) tmem_ld16(s_addr + c, xs);
-          if (RETAIN) {
+          if (kLReg) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) lv[i] = lreg[(c + i) % (RETAIN ? NC : 1)];
+            for (int i = 0; i < 16; ++i) lv[i] = lreg[(c + i) % (kLReg ? NC : 1)];
           } else {
             tmem_ld16(tmem + lane_base + 3 * N + c0 + c, lv);
           }
-          if (!kHold || !RETAIN) tmem_ld_wait();
+          if (!kHold || !kLReg) tmem_ld_wait();
           const float* x = xs + (kHold ? c : 0);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -561,13 +567,22 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
             const float pr = (ok && !over && mr != kNegInf) ? fast_exp2(xl - mr) : 0.f;
             pk[i] = pr;
             lv[i] = undo ? lv[i] - pr : lv[i] + pr;
-            if (kPMN || undo) continue;
-            if (FP8)
-              *reinterpret_cast<__half*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
-                  __float2half_rn(pr * vsc);
-            else
-              *reinterpret_cast<__nv_bfloat16*>(pt + (c + i) * 128 + xoff[(c0 + c + i) & 7]) =
-                  __float2bfloat16_rn(pr);
+          }
+          if (!kPMN && !undo) {
+            // P^T K-major: the two keys of a lane pair share each row's 4-byte
+            // word -- the even lane writes rows c+2u, the odd lane rows c+2u+1
+            const bool odd = (lane & 1) != 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float lo = FP8 ? pk[2 * u] * vsc : pk[2 * u];
+              const float hi = FP8 ? pk[2 * u + 1] * vsc : pk[2 * u + 1];
+              const float other = __shfl_xor_sync(0xffffffffu, odd ? lo : hi, 1);
+              const uint32_t w = FP8 ? (odd ? pack_f16(other, hi) : pack_f16(lo, other))
+                                     : (odd ? pack_bf16(other, hi) : pack_bf16(lo, other));
+              const int r = c + 2 * u + (odd ? 1 : 0);
+              *reinterpret_cast<uint32_t*>(pt + r * 128 + ((kchunk ^ (uint32_t)((c0 + r) & 7)) << 4) +
+                                           kpair) = w;
+            }
           }
           if (kPMN && !undo) {  // this key's 16 rows c0+c .. c0+c+15: two packed 16-byte chunks
             uint32_t w[8];
@@ -582,13 +597,13 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
             *reinterpret_cast<uint4*>(prow + (((ch + 1) ^ (keyrow & 7)) << 4)) =
                 make_uint4(w[4], w[5], w[6], w[7]);
           }
-          if (RETAIN) {
+          if (kLReg) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) lreg[(c + i) % (RETAIN ? NC : 1)] = lv[i];
-            tmem_st16(s_addr + c, pk);
+            for (int i = 0; i < 16; ++i) lreg[(c + i) % (kLReg ? NC : 1)] = lv[i];
           } else {
             tmem_st16(tmem + lane_base + 3 * N + c0 + c, lv);
           }
+          if (RETAIN && !undo) tmem_st16(s_addr + c, pk);
         }
         return over_any;
       };
@@ -655,9 +670,9 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
 #pragma unroll
         for (int c = 0; c < NC; c += 16) {
           float v[16];
-          if (RETAIN) {
+          if (kLReg) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) lreg[(c + i) % (RETAIN ? NC : 1)] *= corr[c0 + c + i];
+            for (int i = 0; i < 16; ++i) lreg[(c + i) % (kLReg ? NC : 1)] *= corr[c0 + c + i];
           } else {
             tmem_ld16(tmem + lane_base + 3 * N + c0 + c, v);
             tmem_ld_wait();
@@ -695,9 +710,9 @@ __device__ __forceinline__ void tc_partial_body(const CUtensorMap& kmap, const C
 #pragma unroll
       for (int c = 0; c < NC; c += 16) {
         float v[16];
-        if (RETAIN) {
+        if (kLReg) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = lreg[(c + i) % (RETAIN ? NC : 1)];
+          for (int i = 0; i < 16; ++i) v[i] = lreg[(c + i) % (kLReg ? NC : 1)];
         } else {
           tmem_ld16(tmem + lane_base + 3 * N + c0 + c, v);
           tmem_ld_wait();
@@ -1407,8 +1422,9 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
   }
 }
 
-// Score kernel: warps 0 (TMA), 1 (MMA), score warps 2-5 (plus, for an E4M3
-// cache, converter warps 6-9 writing double-buffered f16 K tiles).
+// Score kernel: warps 0 (TMA), 1 (MMA), score warps 2-9 in two groups of four
+// on alternating tiles (plus, for an E4M3 cache, converter warps 10-13 writing
+// double-buffered f16 K tiles).
 template <int N, int G, bool FP8>
 __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
     attn_tc_score_kernel(const __grid_constant__ CUtensorMap kmap, const FullAttnParams p) {
@@ -1452,7 +1468,7 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
       mbar_init(&k16_full[i], 4);
       mbar_init(&k16_free[i], 1);
     }
-    mbar_init(q_ready, 4);
+    mbar_init(q_ready, 8);
     fence_mbar_init();
   }
   if (warp == 1 && n_tiles > 0) {
@@ -1498,9 +1514,9 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
         tc_commit(FP8 ? &k16_free[bb] : &kv_empty[s]);
       }
     }
-  } else if (FP8 && warp >= 6) {
-    // ---- E4M3 -> f16 converters: warp 6 + i converts key rows 32i .. 32i+31
-    const int i = warp - 6;
+  } else if (FP8 && warp >= 10) {
+    // ---- E4M3 -> f16 converters: warp 10 + i converts key rows 32i .. 32i+31
+    const int i = warp - 10;
     for (int n = 0; n < n_tiles; ++n) {
       const int s = n % S, bb = n & 1;
       if (!mbar_wait(&kv_full[s], (n / S) & 1)) break;
@@ -1517,23 +1533,24 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
   } else {
     // ---- score warps: stage Q (for the tensor cores), the group's (m, l)
     //      partials, clear the histograms; then lse (base 2) of the group's rows
+    constexpr int kSc = 256;  // score threads
     const int st = threadIdx.x - 64;
     if (n_tiles > 0) {
-      tc_stage_q<N, FP8>(p, b, t0, smem + SM::kSQOff, st, 128);
+      tc_stage_q<N, FP8>(p, b, t0, smem + SM::kSQOff, st, kSc);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
     }
     if (!p.lse_in) {
       const float2* ml_g = p.part_ml + (long long)grp * ns * N;
-      for (int u = st; u < N * ns; u += 128) {
+      for (int u = st; u < N * ns; u += kSc) {
         const int sp = u / N, r = u % N;
         ml_s[r * ns + sp] = ml_g[(long long)sp * N + r];
       }
     }
-    for (int u = st; u < G * kHistBins; u += 128) hist_s[u] = 0u;
-    softmax_sync<128>();
-    for (int r = st; r < N; r += 128) {
+    for (int u = st; u < G * kHistBins; u += kSc) hist_s[u] = 0u;
+    softmax_sync<kSc>();
+    for (int r = st; r < N; r += kSc) {
       if (p.lse_in) {  // the normaliser over the whole context (context-parallel slice)
         const int t = t0 + r / kH;
         lse2_s[r] = t < p.T ? p.lse_in[((long long)b * p.T + t) * p.H + r % kH] * kLog2e : 0.f;
@@ -1549,22 +1566,23 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
         }
       lse2_s[r] = M + log2f(lt);
     }
-    softmax_sync<128>();
+    softmax_sync<kSc>();
     const int wq = warp & 3;
+    const int half = (warp - 2) >> 2;  // this group's tiles: half, half + 2, ...
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const int keyrow = wq * 32 + lane;
     auto load_ks = [&](int n) {
       const long long jn = k_lo + (long long)n * kTcKeys + keyrow;
       return (FP8 && n < n_tiles && jn < k_hi) ? p.k_scale[(long long)b * p.L + jn] : 0.f;
     };
-    float ks_next = load_ks(0);  // E4M3: one tile ahead of its use
-    for (int n = 0; n < n_tiles; ++n) {
+    float ks_next = load_ks(half);  // E4M3: one tile ahead of its use
+    for (int n = half; n < n_tiles; n += 2) {
       const int bb = n & 1;
       const long long j = k_lo + (long long)n * kTcKeys + keyrow;
       float sl = p.scale_log2;
       if (FP8) {
         sl *= ks_next;
-        ks_next = load_ks(n + 1);
+        ks_next = load_ks(n + 2);
       }
       if (!mbar_wait(&s_full[bb], (n >> 1) & 1)) break;
       tc_fence_after();
@@ -1593,25 +1611,27 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
         hist_inc(hist_s + q * kHistBins, __float_as_uint(acc[q]) >> kHistShift, cand);
       }
     }
-    softmax_sync<128>();
-    for (int u = st; u < G * kHistBins; u += 128) {
+    softmax_sync<kSc>();
+    for (int u = st; u < G * kHistBins; u += kSc) {
       const unsigned cnt = hist_s[u];
       const int t = t0 + u / kHistBins;
       if (cnt && t < p.T) atomicAdd(&p.hist[((long long)b * p.T + t) * kHistBins + (u % kHistBins)], cnt);
     }
     // ---- O and lse of row r, merged by the CTA whose score-split index is r mod
-    //      score_splits: thread st owns element d = st of the row (not with a
-    //      given normaliser: O and lse were produced by the slice's first pass)
-    for (int r = split; r < N && !p.lse_in; r += p.score_splits) {
+    //      score_splits: each group takes every other such row, its thread d
+    //      element d (not with a given normaliser: O and lse were produced by
+    //      the slice's first pass)
+    const int d = st & 127;
+    for (int r = split + half * p.score_splits; r < N && !p.lse_in; r += 2 * p.score_splits) {
       const int t = t0 + r / kH;
       if (t >= p.T) continue;
       const float l2 = lse2_s[r];
       const long long li = ((long long)b * p.T + t) * p.H + r % kH;
-      if (st == 0) {
+      if (d == 0) {
         p.lse[li] = l2 * 0.69314718055994531f;
         if (p.lse_out) p.lse_out[li] = l2 * 0.69314718055994531f;
       }
-      const float* po = p.part_o + ((long long)grp * ns * N + r) * 128 + st;
+      const float* po = p.part_o + ((long long)grp * ns * N + r) * 128 + d;
       float acc = 0.f;
 #pragma unroll 8
       for (int sp = 0; sp < ns; ++sp) {
@@ -1619,7 +1639,7 @@ __global__ void __launch_bounds__(tc_score_threads(FP8), 1)
         const float f = (v.x == kNegInf) ? 0.f : fast_exp2(v.x - l2);
         acc += f * po[(long long)sp * N * 128];
       }
-      p.o[li * 128 + st] = acc;
+      p.o[li * 128 + d] = acc;
     }
   }
   __syncthreads();
