@@ -96,7 +96,8 @@ struct TcSmem {
   static constexpr bool kFusable =
       kHistInV16 ? (kS2Stages * kS2TileBytes <= kRingBytes && kNV16 * kTcTileBytes >= 64 * 1024)
                  : kS2HistOff + 32 * 1024 <= kRingBytes;
-  static constexpr int kSelWorkOff = kQOff - 16 * 1024;  // counters, list offsets
+  // counters (2048), list offsets, the lower splits' counters (2048 + 512)
+  static constexpr int kSelWorkOff = kQOff - 24 * 1024;
   static constexpr int kSelCap = kSelWorkOff / 4;        // list entries held in smem
   // score kernel
   static constexpr int kSStages = (FP8 || N == 32) ? 4 : 3;
@@ -988,16 +989,22 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
       }
     }
     softmax_sync<kTcSoftmax>();
-    for (int r = st; r < N; r += kTcSoftmax) {
+    {  // eight threads per row, each over every eighth split, then a shuffle combine
+      static_assert(N * 8 == kTcSoftmax, "eight threads per row");
+      const int r = st >> 3, sub = st & 7;
       float M = kNegInf;
-      for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, ml_s[r * ns + sp].x);
+      for (int sp = sub; sp < ns; sp += 8) M = fmaxf(M, ml_s[r * ns + sp].x);
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
       float lt = 0.f;
       if (M != kNegInf)
-        for (int sp = 0; sp < ns; ++sp) {
+        for (int sp = sub; sp < ns; sp += 8) {
           const float2 v = ml_s[r * ns + sp];
           lt += v.x == kNegInf ? 0.f : v.y * fast_exp2(v.x - M);
         }
-      lse2_s[r] = M + log2f(lt);
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
+      if (sub == 0) lse2_s[r] = M + log2f(lt);
     }
     softmax_sync<kTcSoftmax>();
     // RETAIN: TMEM holds p = 2^(x - m_ref(tile)); f[tile][r] = 2^(m_ref(tile) - lse)
@@ -1170,6 +1177,9 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
     unsigned* list_s = reinterpret_cast<unsigned*>(smem);                 // the row's b1 list
     unsigned* h = reinterpret_cast<unsigned*>(smem + SM::kSelWorkOff);    // 2048 counters
     int* off_s = reinterpret_cast<int*>(smem + SM::kSelWorkOff + 8192);   // [ns + 1] list offsets
+    // the same digit counts of the list elements before this split's slice
+    unsigned* hp2 = reinterpret_cast<unsigned*>(smem + SM::kSelWorkOff + 12288);  // 2048
+    unsigned* hp3 = hp2 + 2048;                                                   // 512
     __shared__ int s_red[2][16];
     auto row_of = [&](int q) { return (long long)b * p.T + t0 + q; };
     auto nc_of = [&](int q) { return p.qpos0 + t0 + q - p.window + 1; };
@@ -1292,7 +1302,8 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
             s_base[1] = in_ex;
           }
         }
-        for (int e = threadIdx.x; e < 2048; e += kThreads) h[e] = 0u;
+        for (int e = threadIdx.x; e < 2048; e += kThreads) h[e] = hp2[e] = 0u;
+        for (int e = threadIdx.x; e < 512; e += kThreads) hp3[e] = 0u;
         __syncthreads();
         const int m = off_s[ns];
         const bool in_smem = m <= SM::kSelCap;
@@ -1320,19 +1331,29 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
         // levels 2 and 3 -- bits [19:9], then [8:0], of the list's elements that
         // share the digits found so far -- as one loop over the same code (it
         // runs once per launch, so every distinct instruction is fetched cold)
+        // The survivors of the lower splits' b1 slices (list elements e < own)
+        // come from the same passes: hp2 / hp3 count their digits, and those
+        // above each level's bin are above tau.
+        const int own = s_base[1];
         unsigned tau = (unsigned)s_prefix[q];
         int need_tau = s_need[q];
+        int a = 0;
 #pragma unroll 1
         for (int lvl = 0; lvl < 2; ++lvl) {
           const int shift = lvl == 0 ? 9 : 0;
           const int kept = lvl == 0 ? 20 : 9;   // bits above the digit: those found so far
+          const int nb = lvl == 0 ? 2048 : 512;
+          unsigned* hp = lvl == 0 ? hp2 : hp3;
           if (lvl == 1) {
             for (int e = threadIdx.x; e < 512; e += kThreads) h[e] = 0u;
             __syncthreads();
           }
           for (int e = threadIdx.x; e < m; e += kThreads) {
             const unsigned v = val(e);
-            hist_inc(h, (v >> shift) & (lvl == 0 ? 2047u : 511u), (v >> kept) == tau);
+            const unsigned bin = (v >> shift) & (unsigned)(nb - 1);
+            const bool in = (v >> kept) == tau;
+            hist_inc(h, bin, in);
+            hist_inc(hp, bin, in && e < own);
           }
           __syncthreads();
           if (warp == 0) {
@@ -1340,19 +1361,13 @@ __global__ void __launch_bounds__(tc_partial_threads(FP8), 1)
             else sel_find_bin_warp<512>(h, need_tau, s_res);
           }
           __syncthreads();
+          for (int e = threadIdx.x; e < nb; e += kThreads) a += e > s_res[0] ? (int)hp[e] : 0;
           tau = (tau << (lvl == 0 ? 11 : 9)) | (unsigned)s_res[0];
           need_tau = s_res[1];
         }
-        // survivors of the lower splits' b1 slices: above tau, and ties
-        const int own = s_base[1];
-        int a = 0, tie = 0;
-        for (int e = threadIdx.x; e < own; e += kThreads) {
-          const unsigned v = val(e);
-          a += v > tau;
-          tie += v == tau;
-        }
-        int a_tot, tie_tot;
-        block_sum2(a, tie, a_tot, tie_tot);
+        int a_tot, unused;
+        block_sum2(a, 0, a_tot, unused);
+        const int tie_tot = (int)hp3[tau & 511u];
         // this split's survivors, per warp-contiguous part: v > tau, v == tau
         const int n = nseg_of(q);
         const int wseg = (n + W - 1) / W;
