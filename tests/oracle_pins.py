@@ -5,7 +5,9 @@ CPU casts for the bf16/E4M3 codecs, numpy's float64 matmul for KV Bridging,
 torch float64 softmax/logsumexp for attention, numpy's stable lexsort and a
 brute-force rank count for the selection, closed forms (probabilities sum to
 1 per head, sparse == dense when the context fits the budget, all-equal keys
-tie down to the lowest indices) and a hand-worked fixture under tests/golden.
+tie down to the lowest indices), the selection's invariants on the seeded
+workloads (planted needles and the forced window always selected) and a
+hand-worked fixture under tests/golden.
 
 The checks are plain functions so that the mutation test can run them against
 deliberately broken copies of the oracle.
@@ -343,6 +345,34 @@ def check_golden_worked_block_selection():
     assert idx[:ns].tolist() == g["token_level_topk4"]
 
 
+def check_planted_needles_and_window():
+    # invariants of the selection on the seeded workloads' own inputs: every
+    # planted needle key (k = 4*sqrt(D) times the unit head-sum of a later
+    # query, outside that query's window) is selected for its query, the last
+    # `window` positions are always present, and the set holds min(i + 1,
+    # topk + window) distinct positions <= i
+    from hs2_synth import WORKLOADS, make_attention_inputs
+    for name, kw in (("decode_bf16_32k", dict(B=2, L=2600, n_needles=6, n_sparse=0)),
+                     ("decode_fp8_256k", dict(B=1, L=3100, n_needles=8, n_sparse=0,
+                                              fp8_scale="mantissa")),
+                     ("tiny", dict(T=300, L=1400, n_needles=5, n_sparse=0))):
+        wl = WORKLOADS[name].resized(**kw)
+        inp = make_attention_inputs(wl)
+        assert len(inp.needles) == wl.B * wl.n_needles
+        rows = np.unique([int(b) * wl.T + int(t) for b, _, t in inp.needles] + [0, wl.B * wl.T - 1])
+        r = oracle.full_attn_select(inp.q, inp.k, inp.v, inp.k_scale, inp.v_scale, scale=wl.scale,
+                                    topk=wl.topk, window=wl.window, rows=rows)
+        for k_, row in enumerate(rows):
+            i = wl.L - wl.T + int(row) % wl.T
+            sel = r["idx"][k_, :r["n_sel"][k_]]
+            assert r["n_sel"][k_] == min(i + 1, wl.topk + wl.window)
+            assert len(set(sel.tolist())) == len(sel) and sel.min() >= 0 and sel.max() <= i
+            assert set(range(max(0, i - wl.window + 1), i + 1)) <= set(sel.tolist())
+        for b, j, t in inp.needles:
+            k_ = int(np.searchsorted(rows, int(b) * wl.T + int(t)))
+            assert int(j) in r["idx"][k_, :r["n_sel"][k_]], (name, b, j, t)
+
+
 # ------------------------------------------------------------ sparse layer --
 def check_sparse_equals_dense():
     rng = np.random.default_rng(41)
@@ -398,4 +428,5 @@ ALL_CHECKS = [
     check_golden_worked_example, check_select_blocks_of_one_are_token_level,
     check_select_blocks_bruteforce_rank, check_golden_worked_block_selection,
     check_slice_of_the_whole_cache_is_full_attention, check_slice_vs_torch,
+    check_planted_needles_and_window,
 ]
